@@ -1,0 +1,179 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the single-GPU forward pass of a routed-expert
+ * mixture-of-experts MLP, as hand-written CUDA kernels for sm_100a (B200).
+ *
+ * Pipeline (one CUDA stream, no host synchronisation, no allocation):
+ *
+ *   logits --moe_route--> ids, w --moe_permute--> counts, offsets, row2assign, assign2row
+ *   x (--moe_quantize_x--> xq, sx)            [block-scaled path only]
+ *   x rows gathered by row2assign --moe_grouped_gemm1_swiglu--> act (expert-sorted rows)
+ *   act --moe_grouped_gemm2--> y (expert-sorted rows)
+ *   y, w, assign2row --moe_combine--> out (token order)
+ *   moe_forward runs all of the above on one stream with the caller's workspace.
+ *
+ * Sources of the operations (web pages on routed MoE kernels; none gives an API):
+ *   - TileScale PR #70 (distributed FP8 MegaMoE example), "Design": routing, GEMM1 with
+ *     fused SwiGLU and FP8 requantisation (kernel 1), GEMM2 and the top-k slot reduction
+ *     (kernel 2); the flat m-task queue that replaced a per-tile expert rescan (first
+ *     change listed in the PR description); fp32 per-128-element activation scales.
+ *   - FlashInfer PR #5129 (cuTile BF16 fused MoE), "sorted I/O": GEMM1 writes a padded
+ *     expert-sorted row space that GEMM2 reads contiguously; combine unchanged.
+ *   - FlashInfer PR #6465 (Hopper MXFP4 x FP8 MegaMoE tuning), benchmark setup: MXFP4
+ *     weights with K32 scaling, FP8 activations, BF16 input/output, H=2560, E=512,
+ *     top-k 10, I=640.
+ *   - Liger-Kernel PR #1463 (SM90 MoE), benchmark definition: BF16 routed-expert MoE
+ *     MLP forward, TFLOP/s counted over routed experts only.
+ *
+ * Conventions shared by every entry point
+ *   - Notation: T tokens, H hidden size, I expert intermediate size (GEMM1 width 2I),
+ *     E experts, k experts per token, R = T*k routed rows.
+ *   - Every pointer argument is a DEVICE pointer on the current device unless marked
+ *     "host".  The caller owns every buffer; the library never allocates, frees or
+ *     synchronises on these paths.  All work is enqueued on `stream` (0 = legacy default).
+ *   - Layouts are row-major.  Weights are K-major: W13 is [E][2I][H] with rows [0,I) the
+ *     gate projection and rows [I,2I) the up projection; W2 is [E][H][I].
+ *   - Argument checks run on the host before any launch and return an error without
+ *     enqueuing work.  A failed launch returns MOE_ERR_CUDA.  A device-side bounded wait
+ *     that expires, or a routing id out of range, sets a status word in the workspace;
+ *     moe_get_device_status() reads it.
+ *   - Device pointers must be 16-byte aligned.  BF16 path: H % 64 == 0 and I % 64 == 0.
+ *     Block-scaled path: H % 128 == 0 and I % 128 == 0.  1 <= k <= min(E, 32),
+ *     E <= 1024, 0 <= T and T*k < 2^31.  T == 0 is a valid no-op.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,          /* null pointer, bad enum, k > E, negative T ...      */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,    /* shape outside the preconditions above             */
+  MOE_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned                  */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < moe_workspace_size(shape)              */
+  MOE_ERR_CUDA = 5,                 /* a CUDA runtime/driver call or launch failed       */
+  MOE_ERR_DEVICE_TIMEOUT = 6,       /* device status: a bounded wait expired             */
+  MOE_ERR_DEVICE_BAD_INDEX = 7      /* device status: an expert id outside [0, E)        */
+} moe_status_t;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
+typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_MXFP4 = 1 } moe_dtype_t;
+
+/* Problem description.  score: moe_score_t; renormalize: 1 = divide the k selected
+ * weights by their sum; dtype: moe_dtype_t. */
+typedef struct {
+  int64_t T;
+  int32_t H, I, E, k;
+  int32_t score;
+  int32_t renormalize;
+  int32_t dtype;
+} moe_shape_t;
+
+/* Bytes of device workspace moe_forward needs for `shape` (the stage entry points need
+ * at most the same).  The first 256 bytes hold the device status word; the rest holds
+ * routing metadata, the expert-sorted activations and expert outputs.  Returns 0 for an
+ * invalid shape.  Sizes grow linearly in T*k*(H+I). */
+size_t moe_workspace_size(const moe_shape_t *shape);
+
+/* Zero the status block of a workspace (call once after allocating it). */
+moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Routing (TileScale PR #70 "Design"; FlashInfer PR #6465 top-k 10 workload).
+ * logits: fp32 [T][E] router logits.  ids: int32 [T][k] out, slot j = j-th largest logit,
+ * ties to the lower expert index.  w: fp32 [T][k] out: softmax over the selected logits
+ * when renormalize (else over all E), or sigmoid of the selected logit (renormalised to
+ * sum 1 when renormalize).  No workspace. */
+moe_status_t moe_route(const moe_shape_t *shape, const float *logits, int32_t *ids, float *w,
+                       cudaStream_t stream);
+
+/* Histogram + exclusive prefix sum + stable scatter into the expert-sorted row space
+ * (FlashInfer PR #5129 "sorted I/O").  ids: int32 [T*k] in.  counts: int32 [E] out.
+ * offsets: int32 [E+1] out, offsets[e] = first sorted row of expert e.  row2assign: int32
+ * [R] out, the assignment a = t*k + j held by sorted row r; rows of one expert are in
+ * ascending a.  assign2row: int32 [R] out, its inverse.  ws: workspace (scratch for
+ * per-chunk histograms + status word).  Ids outside [0,E) set MOE_ERR_DEVICE_BAD_INDEX in
+ * the status word and are skipped. */
+moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *counts,
+                         int32_t *offsets, int32_t *row2assign, int32_t *assign2row, void *ws,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Block-scaled path: per token and per 128 consecutive columns, the smallest power of two
+ * s = 2^e (e clamped to [-127,127]) with max|x| <= 448*s, and e4m3 codes of x/s (round to
+ * nearest even, saturating).  TileScale PR #70 "Design" (FP8 E4M3, fp32 per-128 scales).
+ * x: bf16 [T][H].  xq: uint8 e4m3 [T][H] out.  sx: fp32 [T][H/128] out. */
+moe_status_t moe_quantize_x(const moe_shape_t *shape, const uint16_t *x, uint8_t *xq, float *sx,
+                            cudaStream_t stream);
+
+/* One-off weight preparation for the block-scaled path (not on the forward path): MXFP4
+ * per the OCP MX rule, one UE8M0 scale per 32 consecutive K elements: byte =
+ * clamp(floor(log2 amax) - 2 + 127, 0, 254) (0 when amax == 0), codes = e2m1 of
+ * w / 2^(byte-127), round to nearest even, saturating.  FlashInfer PR #6465 (MXFP4 K32).
+ * w: bf16 [rows][K] (K % 32 == 0).  packed: uint8 [rows][K/2] out, element 2i in the low
+ * nibble of byte i.  sf: uint8 [rows][K/32] out. */
+moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const uint16_t *w,
+                                        uint8_t *packed, uint8_t *sf, cudaStream_t stream);
+
+/* Grouped GEMM1 with fused SwiGLU over the expert-sorted rows (TileScale PR #70 kernel 1;
+ * FlashInfer PR #5129 gathered-A GEMM1).  For sorted row r of expert e with token
+ * t = row2assign[r] / k:  act[r][i] = silu(x[t].W13[e][i]) * (x[t].W13[e][I+i]), fp32
+ * accumulation, silu(g) = g / (1 + exp(-g)).
+ *   BF16:  a = x bf16 [T][H]; sa, w13_sf, act_sf unused (may be NULL); w13 bf16 [E][2I][H];
+ *          act bf16 [R][I] out.
+ *   FP8:   a = xq e4m3 [T][H]; sa = sx fp32 [T][H/128]; w13 = MXFP4 [E][2I][H/2];
+ *          w13_sf = UE8M0 [E][2I][H/32]; act = e4m3 [R][I] out, requantised per 1x128
+ *          with the moe_quantize_x rule; act_sf fp32 [R][I/128] out.
+ * offsets: int32 [E+1] from moe_permute.  ws: workspace (status word). */
+moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t *shape, const void *a, const float *sa,
+                                      const int32_t *row2assign, const int32_t *offsets,
+                                      const void *w13, const uint8_t *w13_sf, void *act,
+                                      float *act_sf, void *ws, size_t ws_bytes,
+                                      cudaStream_t stream);
+
+/* Grouped GEMM2 (down projection) over the expert-sorted rows (TileScale PR #70 kernel 2;
+ * FlashInfer PR #5129 sorted-I/O GEMM2).  y[r][o] = act[r].W2[e][o], fp32 accumulation,
+ * bf16 out.
+ *   BF16:  act bf16 [R][I]; w2 bf16 [E][H][I]; act_sf, w2_sf unused.
+ *   FP8:   act e4m3 [R][I] + act_sf fp32 [R][I/128]; w2 MXFP4 [E][H][I/2] + w2_sf UE8M0
+ *          [E][H][I/32].
+ * y: bf16 [R][H] out.  offsets: int32 [E+1].  ws: workspace (status word). */
+moe_status_t moe_grouped_gemm2(const moe_shape_t *shape, const void *act, const float *act_sf,
+                               const int32_t *offsets, const void *w2, const uint8_t *w2_sf,
+                               uint16_t *y, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Top-k weighted combine back to token order (TileScale PR #70, the slot reduction of
+ * kernel 2).  out[t][h] = bf16_rne( sum_{j<k, ascending} w[t][j] * y[assign2row[t*k+j]][h] ),
+ * fp32 sum.  y bf16 [R][H]; w fp32 [T][k]; assign2row int32 [R]; out bf16 [T][H]. */
+moe_status_t moe_combine(const moe_shape_t *shape, const uint16_t *y, const float *w,
+                         const int32_t *assign2row, uint16_t *out, cudaStream_t stream);
+
+/* The whole forward pass on one stream.  x bf16 [T][H]; logits fp32 [T][E]; weights as in
+ * the GEMM entry points for shape->dtype; out bf16 [T][H].  ids_out: optional int32 [T][k]
+ * copy of the routing ids (NULL to skip).  ws: >= moe_workspace_size(shape) bytes,
+ * 256-byte aligned, initialised once with moe_workspace_init. */
+moe_status_t moe_forward(const moe_shape_t *shape, const uint16_t *x, const float *logits,
+                         const void *w13, const uint8_t *w13_sf, const void *w2,
+                         const uint8_t *w2_sf, uint16_t *out, int32_t *ids_out, void *ws,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronise `stream`, read the workspace status word, clear it, and return it
+ * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */
+moe_status_t moe_get_device_status(void *ws, cudaStream_t stream);
+
+/* Static string for a status code (host). */
+const char *moe_status_string(moe_status_t status);
+
+/* Number of kernel launches the last successful call of each entry point enqueued on
+ * this host thread (host). */
+int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,158 @@
+"""Seeded synthetic inputs for the routed-expert MoE MLP workloads.
+
+This module only draws random tensors and builds router logits from them; it holds none
+of the method's arithmetic (no routing, permutation, quantisation or expert math).  Both
+the CUDA path and the CPU oracle consume what it returns.
+
+Workloads (shapes and value recipes):
+  tiny            T=64, H=256, E=8, k=2, I=128, softmax top-2 renormalised.
+  qwen3_30b_a3b   T=8192, H=2048, E=128, k=8, I=768, softmax top-8 renormalised
+                  (shape of the Qwen3-30B-A3B rows of the Liger-Kernel PR #1463 benchmark).
+  llama4_scout    T=8192, H=5120, E=16, k=1, I=8192, sigmoid weight of the top-1 logit
+                  (shape of the Llama 4 Scout rows of the same benchmark).
+  fp8_mxfp4       T in {128, 1024, 8192, 16384}, H=2560, E=512, k=10, I=640, softmax top-10
+                  renormalised, uniform expert load (FlashInfer PR #6465 workload).
+  decode          T in {1, 8, 32, 128, 256}, H=4096, E=8, k=2, I=14336, softmax top-2
+                  renormalised, Zipf(1.2)-skewed expert choice with one expert never chosen.
+
+Values: x ~ N(0,1) bf16; W13 ~ N(0, 1/H) and W2 ~ N(0, 1/I) bf16 (fan-in scaling).
+Router logits:
+  gaussian  logits = fp32(x) @ Wg, Wg ~ N(0, 1/H) fp32 [H, E]: near-uniform load.
+  uniform   assignment a = t*k + j goes to expert a mod E: those k logits are
+            8 + 0.5*U(0,1), the others N(0,1) clipped to [-3, 3]; per-expert counts then
+            differ by at most one.
+  zipf      a seeded permutation gives the experts ranks 1..E; logit = -1.2*ln(rank) +
+            Gumbel(0,1) (so top-k samples k distinct experts with probability ~ rank^-1.2);
+            the rank-E expert gets -1e4 so at least one expert is always empty.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    score: str = "softmax"       # "softmax" | "sigmoid"
+    renorm: bool = True
+    dtype: str = "bf16"          # "bf16" | "fp8_mxfp4"
+    routing: str = "gaussian"    # "gaussian" | "uniform" | "zipf"
+
+    def with_T(self, T: int) -> "Workload":
+        return replace(self, T=T)
+
+    @property
+    def R(self) -> int:
+        return self.T * self.k
+
+    def flops(self) -> float:
+        """Routed-expert FLOPs of one forward pass: 2*H*2I (GEMM1) + 2*I*H (GEMM2) per
+        routed row (router, SwiGLU elementwise and combine excluded)."""
+        return 6.0 * self.T * self.k * self.H * self.I
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 64, 256, 128, 8, 2),
+    "qwen3_30b_a3b": Workload("qwen3_30b_a3b", 8192, 2048, 768, 128, 8),
+    "llama4_scout": Workload("llama4_scout", 8192, 5120, 8192, 16, 1, score="sigmoid",
+                             renorm=False),
+    "fp8_mxfp4": Workload("fp8_mxfp4", 8192, 2560, 640, 512, 10, dtype="fp8_mxfp4",
+                          routing="uniform"),
+    "decode": Workload("decode", 32, 4096, 14336, 8, 2, routing="zipf"),
+}
+FP8_T_SWEEP = (128, 1024, 8192, 16384)
+DECODE_T_SWEEP = (1, 8, 32, 128, 256)
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def make_x(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    g = _gen(seed, device)
+    return torch.randn(wl.T, wl.H, generator=g, device=device).to(torch.bfloat16)
+
+
+def make_weights(wl: Workload, seed: int = 0, device="cpu"):
+    """W13 bf16 [E, 2I, H] (gate rows then up rows) and W2 bf16 [E, H, I], drawn one
+    expert at a time to bound the temporary fp32 memory."""
+    g = _gen(seed + 1, device)
+    w13 = torch.empty(wl.E, 2 * wl.I, wl.H, dtype=torch.bfloat16, device=device)
+    w2 = torch.empty(wl.E, wl.H, wl.I, dtype=torch.bfloat16, device=device)
+    s13, s2 = 1.0 / math.sqrt(wl.H), 1.0 / math.sqrt(wl.I)
+    for e in range(wl.E):
+        w13[e] = (torch.randn(2 * wl.I, wl.H, generator=g, device=device) * s13).to(torch.bfloat16)
+    for e in range(wl.E):
+        w2[e] = (torch.randn(wl.H, wl.I, generator=g, device=device) * s2).to(torch.bfloat16)
+    return w13, w2
+
+
+def make_logits(wl: Workload, x: torch.Tensor, seed: int = 0) -> torch.Tensor:
+    """Router logits fp32 [T, E] per the workload's routing recipe."""
+    device = x.device
+    g = _gen(seed + 2, device)
+    T, E, k = wl.T, wl.E, wl.k
+    if wl.routing == "gaussian":
+        wg = torch.randn(wl.H, E, generator=g, device=device) / math.sqrt(wl.H)
+        prev = torch.backends.cuda.matmul.allow_tf32
+        torch.backends.cuda.matmul.allow_tf32 = False
+        try:
+            return (x.float() @ wg).contiguous()
+        finally:
+            torch.backends.cuda.matmul.allow_tf32 = prev
+    if wl.routing == "uniform":
+        lg = torch.randn(T, E, generator=g, device=device).clamp_(-3.0, 3.0)
+        a = torch.arange(T * k, device=device)
+        tok, ex = a // k, a % E
+        lg[tok, ex] = 8.0 + 0.5 * torch.rand(T * k, generator=g, device=device)
+        return lg.contiguous()
+    if wl.routing == "zipf":
+        perm = torch.randperm(E, generator=g, device=device)
+        rank = torch.empty(E, device=device)
+        rank[perm] = torch.arange(1, E + 1, device=device, dtype=torch.float32)
+        u = torch.rand(T, E, generator=g, device=device).clamp_(1e-12, 1.0 - 1e-7)
+        gumbel = -torch.log(-torch.log(u))
+        lg = -1.2 * torch.log(rank)[None, :] + gumbel
+        lg[:, perm[E - 1]] = -1e4
+        return lg.contiguous()
+    raise ValueError(wl.routing)
+
+
+def make_inputs(wl: Workload, seed: int = 0, device="cpu", weights: bool = True) -> dict:
+    x = make_x(wl, seed, device)
+    out = {"x": x, "logits": make_logits(wl, x, seed)}
+    if weights:
+        out["w13"], out["w2"] = make_weights(wl, seed, device)
+    return out
+
+
+def parity_tokens(T: int, n: int = 256, seed: int = 0) -> np.ndarray:
+    """Seeded token subset for oracle checks at large T: n tokens without replacement,
+    always including 0 and T-1, sorted."""
+    if T <= n:
+        return np.arange(T, dtype=np.int64)
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
+    return np.sort(np.concatenate([[0, T - 1], pick])).astype(np.int64)
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """uint16 bit patterns of a bf16 tensor (moved to host)."""
+    assert t.dtype == torch.bfloat16
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def from_bits(b: np.ndarray) -> torch.Tensor:
+    """bf16 tensor from uint16 bit patterns."""
+    return torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)

@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE MLP forward pass (libmoe.so on B200).
+
+One step = one full forward pass (route -> histogram/prefix-sum/permute -> GEMM1+SwiGLU ->
+GEMM2 -> combine) over one synthetic batch.  Default workload: the Qwen3-30B-A3B-shaped
+BF16 layer at T=8192 (H=2048, E=128, k=8, I=768).  Metric: routed-expert TFLOP/s
+(6*T*k*H*I per step); decode workloads also report us/layer and GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--T T]
+  python bench.py --impl reference ...     # the CPU oracle on the host cores
+
+With N > 1 (launched by torchrun) every rank runs an independent replica of the workload
+(tokens are independent; the path needs no collective), so scaling is weak and the value
+is the sum over ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_routed_histogram_b200 import _capi as C  # noqa: E402
+from mixture_experts_routed_histogram_b200 import inputs as I  # noqa: E402
+
+METRIC = "routed MoE MLP fwd TFLOP/s on 1 B200 at T=8192; µs/layer at decode T"
+# Liger-Kernel PR #1463 benchmark table: Qwen3-30B-A3B-shaped BF16 routed-MoE forward,
+# T=8192, 1 GPU: 599.60 TFLOP/s on B300 (354.38 on H200).  Context only.
+PUBLISHED = {"qwen3_30b_a3b": 599.60}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_init(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload set-up
+
+def build_device_inputs(wl, seed):
+    inp = I.make_inputs(wl, seed, "cuda")
+    return inp
+
+
+def run_stages(shape, wl, inp, ws, bufs, events=None):
+    """One forward pass as separate C-ABI stage calls (same kernels as moe_forward),
+    optionally bracketing each stage with CUDA events for the per-kernel breakdown."""
+    def mark(i):
+        if events is not None:
+            events[i].record()
+    mark(0)
+    C.moe_route(shape, inp["logits"], bufs["ids"], bufs["w"])
+    mark(1)
+    C.moe_permute(shape, bufs["ids"], bufs["counts"], bufs["offsets"], bufs["r2a"], bufs["a2r"], ws)
+    mark(2)
+    C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, bufs["r2a"], bufs["offsets"], inp["w13"],
+                               None, bufs["act"], None, ws)
+    mark(3)
+    C.moe_grouped_gemm2(shape, bufs["act"], None, bufs["offsets"], inp["w2"], None, bufs["y"], ws)
+    mark(4)
+    C.moe_combine(shape, bufs["y"], bufs["w"], bufs["a2r"], bufs["out"])
+    mark(5)
+
+
+STAGES = ["route", "permute", "gemm1_swiglu", "gemm2", "combine"]
+
+
+def algorithmic(wl, counts):
+    """Algorithmic FLOPs and bytes of each stage for the actual per-expert counts."""
+    T, H, Ii, E, k, R = wl.T, wl.H, wl.I, wl.E, wl.k, wl.R
+    ne = int((counts > 0).sum())
+    f = {"gemm1_swiglu": 4.0 * R * H * Ii, "gemm2": 2.0 * R * H * Ii}
+    b = {
+        "route": T * E * 4 + R * 8,
+        "permute": R * 4 * 3 + E * 8,
+        "gemm1_swiglu": ne * 2 * Ii * H * 2 + T * H * 2 + R * Ii * 2 + R * 4,
+        "gemm2": ne * H * Ii * 2 + R * Ii * 2 + R * H * 2,
+        "combine": R * H * 2 + T * H * 2 + R * 8,
+    }
+    # whole-pass bytes without the y round trip (a fused combine could avoid it)
+    b_alg = (ne * 3 * Ii * H * 2 + T * H * 2 * 2 + R * Ii * 2 * 2 + T * E * 4 + R * 16)
+    return f, b, b_alg, ne
+
+
+# ---------------------------------------------------------------- our arm
+
+def bench_ours(args, rank, world, local):
+    wl = I.WORKLOADS[args.workload]
+    if args.T:
+        wl = wl.with_T(args.T)
+    torch.manual_seed(0)
+    inp = build_device_inputs(wl, seed=rank)
+    shape = C.MoeShape.from_workload(wl)
+    ws_bytes = C.moe_workspace_size(shape)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    C.moe_workspace_init(ws)
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device="cuda")
+    R = wl.R
+    bufs = {
+        "ids": torch.empty(wl.T, wl.k, dtype=torch.int32, device="cuda"),
+        "w": torch.empty(wl.T, wl.k, dtype=torch.float32, device="cuda"),
+        "counts": torch.empty(wl.E, dtype=torch.int32, device="cuda"),
+        "offsets": torch.empty(wl.E + 1, dtype=torch.int32, device="cuda"),
+        "r2a": torch.empty(R, dtype=torch.int32, device="cuda"),
+        "a2r": torch.empty(R, dtype=torch.int32, device="cuda"),
+        "act": torch.empty(R, wl.I, dtype=torch.bfloat16, device="cuda"),
+        "y": torch.empty(R, wl.H, dtype=torch.bfloat16, device="cuda"),
+        "out": out,
+    }
+    stream = torch.cuda.current_stream()
+
+    def step():
+        C.moe_forward(shape, inp["x"], inp["logits"], inp["w13"], None, inp["w2"], None, out,
+                      None, ws)
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = C.moe_last_launch_count()
+
+    # ---- timed region: K forward passes through moe_forward
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    st = C.moe_get_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {C.moe_status_string(st)}")
+
+    # ---- per-kernel breakdown (stage calls, events on the launching stream)
+    run_stages(shape, wl, inp, ws, bufs)
+    torch.cuda.synchronize()
+    acc = np.zeros(len(STAGES))
+    for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+        run_stages(shape, wl, inp, ws, bufs, ev)
+        torch.cuda.synchronize()
+        acc += [ev[i].elapsed_time(ev[i + 1]) for i in range(len(STAGES))]
+    stage_ms = acc / args.steps
+    counts = bufs["counts"].cpu().numpy()
+    flops_s, bytes_s, b_alg, ne = algorithmic(wl, counts)
+
+    # ---- end to end through the public API: pinned host input -> device -> host output
+    x_h = inp["x"].cpu().pin_memory()
+    lg_h = inp["logits"].cpu().pin_memory()
+    out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(inp["x"])
+    lg_d = torch.empty_like(inp["logits"])
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        C.moe_forward(shape, x_d, lg_d, inp["w13"], None, inp["w2"], None, out, None, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3) / args.steps, world)
+
+    flops = wl.flops()
+    tflops = flops * world / (ms_max * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    # dominant kernel: the stage with the largest measured share
+    dom = int(np.argmax(stage_ms))
+    dname = STAGES[dom]
+    t_ker = stage_ms[dom] * 1e-3
+    if dname in flops_s:
+        t_tensor = flops_s[dname] / (pk["bf16_tflops"] * 1e12)
+        t_hbm = bytes_s[dname] / (pk["hbm_gbs"] * 1e9)
+    else:
+        t_tensor, t_hbm = 0.0, 1.0
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": flops_s[dname] / t_ker / 1e12,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": bytes_s[dname] / t_ker / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dname
+    roof["peak_source"] = f"{pk_kind} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"
+
+    result = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 4),
+        "us_per_layer": round(ms_max * 1e3, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": (round(tflops / world / PUBLISHED[wl.name], 4)
+                        if wl.name in PUBLISHED and wl.T == 8192 else None),
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, random-init)",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   "score": wl.score, "routing": wl.routing, "parallelism": f"replicas x{world}",
+                   "nonempty_experts": ne,
+                   "l2": "inputs larger than L2 (weights %.2f GB re-read every step)" %
+                         ((3 * wl.E * wl.I * wl.H * 2) / 1e9)},
+        "hbm_gbs_alg": round(b_alg / (ms_max * 1e-3) / 1e9, 1),
+        "hbm_frac_alg": round(b_alg / (ms_max * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+        "roofline": roof,
+        "stages_ms": {s: round(float(v), 4) for s, v in zip(STAGES, stage_ms)},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
+                "d2h_bytes_per_step": out_h.numel() * 2},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, inp, budget_s=args.cpu_budget)
+    return result
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline only)
+
+def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
+    """Time the fp64 oracle on a bounded sample of the same workload: routing + permutation
+    on all T tokens, the expert MLP on a token subset sized for the budget; TFLOP/s over
+    the subset's routed FLOPs.  Baseline only."""
+    import oracle
+    x = I.bits(inp["x"])
+    lg = inp["logits"].cpu().numpy()
+    w13 = I.bits(inp["w13"])
+    w2 = I.bits(inp["w2"])
+    score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
+    t0 = time.perf_counter()
+    ids, w = oracle.route(lg, wl.k, score, wl.renorm)
+    oracle.permute(ids, wl.E)
+    t_route = time.perf_counter() - t0
+    # probe the per-token cost on a few tokens, then size the sample for the budget
+    probe = I.parity_tokens(wl.T, 4, seed=1)
+    t0 = time.perf_counter()
+    oracle.forward_bf16(x, ids, w, w13, w2, probe)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    n = int(max(4, min(wl.T, (budget_s - t_route) / max(per_tok, 1e-6)))) if T_sample is None else T_sample
+    toks = I.parity_tokens(wl.T, n, seed=2)
+    t0 = time.perf_counter()
+    oracle.forward_bf16(x, ids, w, w13, w2, toks)
+    t_mlp = time.perf_counter() - t0
+    # scale the subset time to all T tokens; routing/permutation counted once
+    t_full = t_route + t_mlp * wl.T / len(toks)
+    return {"value": round(wl.flops() / t_full / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"route+permute on all {wl.T} tokens ({t_route:.2f}s); expert MLP on "
+                      f"{len(toks)} of {wl.T} tokens ({t_mlp:.2f}s), extrapolated x{wl.T / len(toks):.1f}",
+            "seconds_measured": round(t_route + t_mlp, 2)}
+
+
+def bench_reference(args, rank, world):
+    """The oracle as the reference arm: each step is the oracle on a bounded token sample
+    of the same workload (fp64, host cores)."""
+    wl = I.WORKLOADS[args.workload]
+    if args.T:
+        wl = wl.with_T(args.T)
+    if rank != 0:
+        return None
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = I.make_inputs(wl, 0, dev)
+    import oracle
+    x = I.bits(inp["x"])
+    lg = inp["logits"].cpu().numpy()
+    w13 = I.bits(inp["w13"])
+    w2 = I.bits(inp["w2"])
+    score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
+    ids, w = oracle.route(lg, wl.k, score, wl.renorm)
+    probe = I.parity_tokens(wl.T, 4, seed=1)
+    t0 = time.perf_counter()
+    oracle.forward_bf16(x, ids, w, w13, w2, probe)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    per_step_budget = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    n = int(max(2, min(wl.T, per_step_budget / max(per_tok, 1e-6))))
+    times = []
+    for s in range(args.warmup + args.steps):
+        toks = I.parity_tokens(wl.T, n, seed=10 + s)
+        t0 = time.perf_counter()
+        oracle.route(lg, wl.k, score, wl.renorm)
+        oracle.forward_bf16(x, ids, w, w13, w2, toks)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    sec = float(np.mean(times))
+    flops = 6.0 * n * wl.k * wl.H * wl.I
+    val = flops / sec / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": f"{n} of {wl.T} tokens per step (routing on all T)"},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3_30b_a3b", choices=list(I.WORKLOADS))
+    ap.add_argument("--T", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_init(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = bench_reference(args, rank, world)
+        else:
+            res = bench_ours(args, rank, world, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

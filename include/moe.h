@@ -47,6 +47,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -79,17 +85,17 @@ typedef struct {
  * at most the same).  The first 256 bytes hold the device status word; the rest holds
  * routing metadata, the expert-sorted activations and expert outputs.  Returns 0 for an
  * invalid shape.  Sizes grow linearly in T*k*(H+I). */
-size_t moe_workspace_size(const moe_shape_t *shape);
+MOE_API size_t moe_workspace_size(const moe_shape_t *shape);
 
 /* Zero the status block of a workspace (call once after allocating it). */
-moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
+MOE_API moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Routing (TileScale PR #70 "Design"; FlashInfer PR #6465 top-k 10 workload).
  * logits: fp32 [T][E] router logits.  ids: int32 [T][k] out, slot j = j-th largest logit,
  * ties to the lower expert index.  w: fp32 [T][k] out: softmax over the selected logits
  * when renormalize (else over all E), or sigmoid of the selected logit (renormalised to
  * sum 1 when renormalize).  No workspace. */
-moe_status_t moe_route(const moe_shape_t *shape, const float *logits, int32_t *ids, float *w,
+MOE_API moe_status_t moe_route(const moe_shape_t *shape, const float *logits, int32_t *ids, float *w,
                        cudaStream_t stream);
 
 /* Histogram + exclusive prefix sum + stable scatter into the expert-sorted row space
@@ -99,7 +105,7 @@ moe_status_t moe_route(const moe_shape_t *shape, const float *logits, int32_t *i
  * ascending a.  assign2row: int32 [R] out, its inverse.  ws: workspace (scratch for
  * per-chunk histograms + status word).  Ids outside [0,E) set MOE_ERR_DEVICE_BAD_INDEX in
  * the status word and are skipped. */
-moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *counts,
+MOE_API moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *counts,
                          int32_t *offsets, int32_t *row2assign, int32_t *assign2row, void *ws,
                          size_t ws_bytes, cudaStream_t stream);
 
@@ -107,7 +113,7 @@ moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, int32_t *
  * s = 2^e (e clamped to [-127,127]) with max|x| <= 448*s, and e4m3 codes of x/s (round to
  * nearest even, saturating).  TileScale PR #70 "Design" (FP8 E4M3, fp32 per-128 scales).
  * x: bf16 [T][H].  xq: uint8 e4m3 [T][H] out.  sx: fp32 [T][H/128] out. */
-moe_status_t moe_quantize_x(const moe_shape_t *shape, const uint16_t *x, uint8_t *xq, float *sx,
+MOE_API moe_status_t moe_quantize_x(const moe_shape_t *shape, const uint16_t *x, uint8_t *xq, float *sx,
                             cudaStream_t stream);
 
 /* One-off weight preparation for the block-scaled path (not on the forward path): MXFP4
@@ -116,7 +122,7 @@ moe_status_t moe_quantize_x(const moe_shape_t *shape, const uint16_t *x, uint8_t
  * w / 2^(byte-127), round to nearest even, saturating.  FlashInfer PR #6465 (MXFP4 K32).
  * w: bf16 [rows][K] (K % 32 == 0).  packed: uint8 [rows][K/2] out, element 2i in the low
  * nibble of byte i.  sf: uint8 [rows][K/32] out. */
-moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const uint16_t *w,
+MOE_API moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const uint16_t *w,
                                         uint8_t *packed, uint8_t *sf, cudaStream_t stream);
 
 /* Grouped GEMM1 with fused SwiGLU over the expert-sorted rows (TileScale PR #70 kernel 1;
@@ -129,7 +135,7 @@ moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const uint16_t 
  *          w13_sf = UE8M0 [E][2I][H/32]; act = e4m3 [R][I] out, requantised per 1x128
  *          with the moe_quantize_x rule; act_sf fp32 [R][I/128] out.
  * offsets: int32 [E+1] from moe_permute.  ws: workspace (status word). */
-moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t *shape, const void *a, const float *sa,
+MOE_API moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t *shape, const void *a, const float *sa,
                                       const int32_t *row2assign, const int32_t *offsets,
                                       const void *w13, const uint8_t *w13_sf, void *act,
                                       float *act_sf, void *ws, size_t ws_bytes,
@@ -142,35 +148,43 @@ moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t *shape, const void *a, c
  *   FP8:   act e4m3 [R][I] + act_sf fp32 [R][I/128]; w2 MXFP4 [E][H][I/2] + w2_sf UE8M0
  *          [E][H][I/32].
  * y: bf16 [R][H] out.  offsets: int32 [E+1].  ws: workspace (status word). */
-moe_status_t moe_grouped_gemm2(const moe_shape_t *shape, const void *act, const float *act_sf,
+MOE_API moe_status_t moe_grouped_gemm2(const moe_shape_t *shape, const void *act, const float *act_sf,
                                const int32_t *offsets, const void *w2, const uint8_t *w2_sf,
                                uint16_t *y, void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Top-k weighted combine back to token order (TileScale PR #70, the slot reduction of
  * kernel 2).  out[t][h] = bf16_rne( sum_{j<k, ascending} w[t][j] * y[assign2row[t*k+j]][h] ),
  * fp32 sum.  y bf16 [R][H]; w fp32 [T][k]; assign2row int32 [R]; out bf16 [T][H]. */
-moe_status_t moe_combine(const moe_shape_t *shape, const uint16_t *y, const float *w,
+MOE_API moe_status_t moe_combine(const moe_shape_t *shape, const uint16_t *y, const float *w,
                          const int32_t *assign2row, uint16_t *out, cudaStream_t stream);
 
 /* The whole forward pass on one stream.  x bf16 [T][H]; logits fp32 [T][E]; weights as in
  * the GEMM entry points for shape->dtype; out bf16 [T][H].  ids_out: optional int32 [T][k]
  * copy of the routing ids (NULL to skip).  ws: >= moe_workspace_size(shape) bytes,
  * 256-byte aligned, initialised once with moe_workspace_init. */
-moe_status_t moe_forward(const moe_shape_t *shape, const uint16_t *x, const float *logits,
+MOE_API moe_status_t moe_forward(const moe_shape_t *shape, const uint16_t *x, const float *logits,
                          const void *w13, const uint8_t *w13_sf, const void *w2,
                          const uint8_t *w2_sf, uint16_t *out, int32_t *ids_out, void *ws,
                          size_t ws_bytes, cudaStream_t stream);
 
 /* Synchronise `stream`, read the workspace status word, clear it, and return it
  * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */
-moe_status_t moe_get_device_status(void *ws, cudaStream_t stream);
+MOE_API moe_status_t moe_get_device_status(void *ws, cudaStream_t stream);
 
 /* Static string for a status code (host). */
-const char *moe_status_string(moe_status_t status);
+MOE_API const char *moe_status_string(moe_status_t status);
+
+/* Test hooks for failure detection (host).  moe_debug_set_wait_limit_ns sets the bound on
+ * every device-side wait (default 4 s; 0 restores the default).  moe_debug_inject_stall(1)
+ * makes CTA 0 of every following grouped-GEMM launch leave its first pipeline stage
+ * unfilled, so that its consumer's bounded wait expires, the kernel unwinds and the status
+ * word reads MOE_ERR_DEVICE_TIMEOUT; outputs of such calls are undefined.  (0 = off.) */
+MOE_API void moe_debug_set_wait_limit_ns(uint64_t ns);
+MOE_API void moe_debug_inject_stall(int on);
 
 /* Number of kernel launches the last successful call of each entry point enqueued on
  * this host thread (host). */
-int moe_last_launch_count(void);
+MOE_API int moe_last_launch_count(void);
 
 #ifdef __cplusplus
 }

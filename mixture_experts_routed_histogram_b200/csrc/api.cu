@@ -1,0 +1,309 @@
+// api.cu -- the C ABI declared in include/moe.h: host-side argument checks, workspace
+// carving and the ordering of the kernels on the caller's stream.  No allocation, no
+// synchronisation (except moe_get_device_status, which exists to synchronise).
+#include <stdint.h>
+#include <stdlib.h>
+
+#include "kernels.h"
+#include "moe.h"
+
+namespace {
+
+thread_local int g_last_launches = 0;
+uint64_t g_wait_limit_ns = 4000000000ull;  // 4 s per bounded device wait
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace regions (byte offsets from the workspace base).
+struct WsLayout {
+  size_t status, ids, w, counts, offsets, r2a, a2r, scratch, xq, sx, act, act_sf, y, total;
+};
+
+WsLayout layout(const moe_shape_t& s) {
+  const size_t T = static_cast<size_t>(s.T), R = T * s.k, H = s.H, I = s.I, E = s.E;
+  const bool fp8 = s.dtype == MOE_DTYPE_FP8_MXFP4;
+  WsLayout L{};
+  size_t o = 0;
+  L.status = o; o += kStatusBytes;
+  L.ids = o; o = up(o + 4 * R);
+  L.w = o; o = up(o + 4 * R);
+  L.counts = o; o = up(o + 4 * E);
+  L.offsets = o; o = up(o + 4 * (E + 1));
+  L.r2a = o; o = up(o + 4 * R);
+  L.a2r = o; o = up(o + 4 * R);
+  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(R), s.E));
+  L.xq = o; o = up(o + (fp8 ? T * H : 0));
+  L.sx = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
+  L.act = o; o = up(o + (fp8 ? R * I : 2 * R * I));
+  L.act_sf = o; o = up(o + (fp8 ? 4 * R * (I / 128) : 0));
+  L.y = o; o = up(o + 2 * R * H);
+  L.total = o;
+  return L;
+}
+
+moe_status_t check_shape(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E <= 0 || s->k <= 0) return MOE_ERR_INVALID_ARG;
+  if ((s->score != MOE_SCORE_SOFTMAX && s->score != MOE_SCORE_SIGMOID) ||
+      (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_FP8_MXFP4) ||
+      (s->renormalize != 0 && s->renormalize != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->k > moe::kMaxTopK || s->E > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->T * static_cast<int64_t>(s->k) >= (static_cast<int64_t>(1) << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int q = s->dtype == MOE_DTYPE_BF16 ? 64 : 128;
+  if (s->H % q != 0 || s->I % q != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                    \
+  do {                                   \
+    moe_status_t st_ = (expr);           \
+    if (st_ != MOE_OK) return st_;       \
+  } while (0)
+
+moe_status_t need_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  return MOE_OK;
+}
+
+moe::GemmProblem problem(const moe_shape_t& s) {
+  moe::GemmProblem p{};
+  p.T = s.T;
+  p.R = s.T * s.k;
+  p.H = s.H;
+  p.I = s.I;
+  p.E = s.E;
+  p.k = s.k;
+  p.wait_limit_ns = g_wait_limit_ns;
+  return p;
+}
+
+int* status_word(void* ws) { return reinterpret_cast<int*>(ws); }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return layout(*shape).total;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_last_launches = 0;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_MISALIGNED;
+  if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  g_last_launches = 1;
+  return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, stream));
+}
+
+moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* ids, float* w,
+                       cudaStream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_shape(shape));
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({logits, ids, w}));
+  int n = 0;
+  cudaError_t e = moe::launch_route(logits, ids, w, shape->T, shape->E, shape->k, shape->score,
+                                    shape->renormalize, stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
+                         int32_t* offsets, int32_t* row2assign, int32_t* assign2row, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(need_ptrs({counts, offsets, ws}));
+  const int64_t R = shape->T * shape->k;
+  if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
+  const WsLayout L = layout(*shape);
+  if (ws_bytes < L.scratch + moe::permute_scratch_bytes(R, shape->E))
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int n = 0;
+  cudaError_t e = moe::launch_permute(ids, R, shape->E, counts, offsets, row2assign, assign2row,
+                                      at<int32_t>(ws, L.scratch), status_word(ws), stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_quantize_x(const moe_shape_t* shape, const uint16_t* x, uint8_t* xq, float* sx,
+                            cudaStream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_shape(shape));
+  if (shape->H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({x, xq, sx}));
+  int n = 0;
+  cudaError_t e = moe::launch_quant_x(x, xq, sx, shape->T, shape->H, stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const uint16_t* w,
+                                        uint8_t* packed, uint8_t* sf, cudaStream_t stream) {
+  g_last_launches = 0;
+  if (rows < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (K % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!w || !packed || !sf) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(packed)) return MOE_ERR_MISALIGNED;
+  int n = 0;
+  cudaError_t e = moe::launch_quant_w_mxfp4(w, packed, sf, rows, K, stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t* shape, const void* a, const float* sa,
+                                      const int32_t* row2assign, const int32_t* offsets,
+                                      const void* w13, const uint8_t* w13_sf, void* act,
+                                      float* act_sf, void* ws, size_t ws_bytes,
+                                      cudaStream_t stream) {
+  g_last_launches = 0;
+  (void)sa; (void)w13_sf; (void)act_sf;
+  MOE_TRY(check_shape(shape));
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
+  MOE_TRY(need_ptrs({offsets, ws}));
+  if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({a, row2assign, w13, act}));
+  int n = 0;
+  cudaError_t e = moe::launch_gemm1_bf16(problem(*shape), static_cast<const uint16_t*>(a),
+                                         row2assign, offsets, static_cast<const uint16_t*>(w13),
+                                         static_cast<uint16_t*>(act), status_word(ws), stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_grouped_gemm2(const moe_shape_t* shape, const void* act, const float* act_sf,
+                               const int32_t* offsets, const void* w2, const uint8_t* w2_sf,
+                               uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_last_launches = 0;
+  (void)act_sf; (void)w2_sf;
+  MOE_TRY(check_shape(shape));
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
+  MOE_TRY(need_ptrs({offsets, ws}));
+  if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({act, w2, y}));
+  int n = 0;
+  cudaError_t e = moe::launch_gemm2_bf16(problem(*shape), static_cast<const uint16_t*>(act),
+                                         offsets, static_cast<const uint16_t*>(w2), y,
+                                         status_word(ws), stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_combine(const moe_shape_t* shape, const uint16_t* y, const float* w,
+                         const int32_t* assign2row, uint16_t* out, cudaStream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_shape(shape));
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({y, w, assign2row, out}));
+  int n = 0;
+  cudaError_t e = moe::launch_combine(y, w, assign2row, out, shape->T, shape->H, shape->k, stream,
+                                      &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const float* logits,
+                         const void* w13, const uint8_t* w13_sf, const void* w2,
+                         const uint8_t* w2_sf, uint16_t* out, int32_t* ids_out, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
+  g_last_launches = 0;
+  (void)w13_sf; (void)w2_sf;
+  MOE_TRY(check_shape(shape));
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_MISALIGNED;
+  const WsLayout L = layout(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (shape->T == 0) return MOE_OK;
+  MOE_TRY(need_ptrs({x, logits, w13, w2, out}));
+  if (ids_out && !aligned16(ids_out)) return MOE_ERR_MISALIGNED;
+
+  const int64_t T = shape->T, R = T * shape->k;
+  int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
+  float* w = at<float>(ws, L.w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* r2a = at<int32_t>(ws, L.r2a);
+  int32_t* a2r = at<int32_t>(ws, L.a2r);
+  uint16_t* act = at<uint16_t>(ws, L.act);
+  uint16_t* y = at<uint16_t>(ws, L.y);
+  int* status = status_word(ws);
+  const moe::GemmProblem p = problem(*shape);
+  int n = 0;
+  cudaError_t e;
+  if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->score,
+                             shape->renormalize, stream, &n)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((e = moe::launch_permute(ids, R, shape->E, counts, offsets, r2a, a2r,
+                               at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+                                  status, stream, &n)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((e = moe::launch_gemm2_bf16(p, act, offsets, static_cast<const uint16_t*>(w2), y, status,
+                                  stream, &n)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((e = moe::launch_combine(y, w, a2r, out, T, shape->H, shape->k, stream, &n)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  g_last_launches = n;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
+  g_last_launches = 0;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  int host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host != 0 && cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status_t>(host);
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_MISALIGNED: return "misaligned pointer";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_BAD_INDEX: return "expert id out of range";
+  }
+  return "unknown status";
+}
+
+int moe_last_launch_count(void) { return g_last_launches; }
+
+void moe_debug_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 4000000000ull; }
+
+void moe_debug_inject_stall(int on) { moe::g_inject_stall = on ? 1 : 0; }
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+// combine_quant.cu -- the HBM-bound elementwise stages: top-k weighted combine, the 1x128
+// e4m3 activation quantiser and the MXFP4 weight preparation.
+//
+// Combine: TileScale PR #70 (distributed FP8 MegaMoE), kernel 2 "L2 + scatter + reduce":
+// the expert outputs of a token's k slots are summed with their routing weights in a
+// fixed slot order.  Here the k rows are read from the expert-sorted y through
+// assign2row (FlashInfer PR #5129, sorted I/O: the combine itself is unchanged).
+//
+// Activation quantiser: TileScale PR #70, "Design": FP8 E4M3 with fp32 scales per 128
+// elements; the scale is the smallest power of two keeping the group's amax within 448
+// (so it is also an exact UE8M0 value for the block-scaled MMA).
+//
+// Weight preparation: FlashInfer PR #6465, MXFP4 weights with K32 UE8M0 scaling; the
+// scale follows the OCP MX rule 2^(floor(log2 amax) - 2).
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const uint16_t* __restrict__ y, const float* __restrict__ w,
+                   const int32_t* __restrict__ assign2row, uint16_t* __restrict__ out, int H,
+                   int k) {
+  __shared__ float sw[kMaxTopK];
+  __shared__ int64_t srow[kMaxTopK];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < k) {
+    sw[threadIdx.x] = __ldg(w + t * k + threadIdx.x);
+    srow[threadIdx.x] = static_cast<int64_t>(__ldg(assign2row + t * k + threadIdx.x)) * H;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x * 8; c < H; c += kCombineThreads * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < k; ++j) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(y + srow[j] + c));
+      const float wj = sw[j];
+      acc[0] = fmaf(wj, bf16_lo(v.x), acc[0]);
+      acc[1] = fmaf(wj, bf16_hi(v.x), acc[1]);
+      acc[2] = fmaf(wj, bf16_lo(v.y), acc[2]);
+      acc[3] = fmaf(wj, bf16_hi(v.y), acc[3]);
+      acc[4] = fmaf(wj, bf16_lo(v.z), acc[4]);
+      acc[5] = fmaf(wj, bf16_hi(v.z), acc[5]);
+      acc[6] = fmaf(wj, bf16_lo(v.w), acc[6]);
+      acc[7] = fmaf(wj, bf16_hi(v.w), acc[7]);
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(out + t * H + c) = o;
+  }
+}
+
+// One warp per (token, 128-column group); each lane owns 4 consecutive columns.
+__global__ void __launch_bounds__(256)
+    quant_x_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ xq,
+                   float* __restrict__ sx, int64_t groups, int H) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (gid >= groups) return;
+  const int G = H / 128;
+  const int64_t t = gid / G;
+  const int g = static_cast<int>(gid % G);
+  const int64_t base = t * H + g * 128 + lane * 4;
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(x + base));
+  const float f0 = bf16_lo(v.x), f1 = bf16_hi(v.x), f2 = bf16_lo(v.y), f3 = bf16_hi(v.y);
+  float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const int s = fp8_scale_exponent(amax);
+  const float inv = pow2f(-s);
+  const uint32_t lo = cvt_e4m3x2(f0 * inv, f1 * inv);
+  const uint32_t hi = cvt_e4m3x2(f2 * inv, f3 * inv);
+  *reinterpret_cast<uint32_t*>(xq + base) = lo | (hi << 16);
+  if (lane == 0) sx[t * G + g] = pow2f(s);
+}
+
+// One thread per (row, 32-element group).
+__global__ void __launch_bounds__(256)
+    quant_w_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ packed,
+                   uint8_t* __restrict__ sf, int64_t groups, int K) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (gid >= groups) return;
+  const int G = K / 32;
+  const int64_t r = gid / G;
+  const int g = static_cast<int>(gid % G);
+  const uint4* src = reinterpret_cast<const uint4*>(w + r * K + g * 32);
+  float f[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = __ldg(src + q);
+    f[8 * q + 0] = bf16_lo(v.x); f[8 * q + 1] = bf16_hi(v.x);
+    f[8 * q + 2] = bf16_lo(v.y); f[8 * q + 3] = bf16_hi(v.y);
+    f[8 * q + 4] = bf16_lo(v.z); f[8 * q + 5] = bf16_hi(v.z);
+    f[8 * q + 6] = bf16_lo(v.w); f[8 * q + 7] = bf16_hi(v.w);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  int byte = 0;
+  if (amax > 0.0f) {
+    int e;
+    frexpf(amax, &e);            // amax = m * 2^e, m in [0.5, 1): floor(log2 amax) = e - 1
+    byte = (e - 1) - 2 + 127;
+    byte = byte < 0 ? 0 : (byte > 254 ? 254 : byte);
+  }
+  const float inv = pow2f(127 - byte);
+  uint32_t words[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t wv = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = 8 * q + 2 * b;
+      wv |= cvt_e2m1x2(f[i] * inv, f[i + 1] * inv) << (8 * b);
+    }
+    words[q] = wv;
+  }
+  *reinterpret_cast<uint4*>(packed + r * (K / 2) + g * 16) =
+      make_uint4(words[0], words[1], words[2], words[3]);
+  sf[r * G + g] = static_cast<uint8_t>(byte);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* assign2row,
+                           uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,
+                           int* launches) {
+  if (T == 0) return cudaSuccess;
+  ++*launches;
+  combine_kernel<<<static_cast<unsigned>(T), kCombineThreads, 0, stream>>>(y, w, assign2row, out,
+                                                                           H, k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, int64_t T, int H,
+                           cudaStream_t stream, int* launches) {
+  const int64_t groups = T * (H / 128);
+  if (groups == 0) return cudaSuccess;
+  ++*launches;
+  quant_x_kernel<<<static_cast<unsigned>((groups + 7) / 8), 256, 0, stream>>>(x, xq, sx, groups, H);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_w_mxfp4(const uint16_t* w, uint8_t* packed, uint8_t* sf, int64_t rows,
+                                 int K, cudaStream_t stream, int* launches) {
+  const int64_t groups = rows * (K / 32);
+  if (groups == 0) return cudaSuccess;
+  ++*launches;
+  quant_w_kernel<<<static_cast<unsigned>((groups + 255) / 256), 256, 0, stream>>>(w, packed, sf,
+                                                                                groups, K);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,60 @@
+// kernels.h -- host-side launchers of the CUDA kernels (internal C++ interface used by
+// the C ABI in api.cu).  Every launcher only enqueues work on `stream` and returns the
+// launch error; argument validation is done by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+
+// Routing: ids/w [T][k] from logits [T][E].
+cudaError_t launch_route(const float* logits, int32_t* ids, float* w, int64_t T, int E, int k,
+                         int score, int renorm, cudaStream_t stream, int* launches);
+
+// Histogram / prefix sum / stable scatter.  `scratch` holds the per-chunk histograms.
+size_t permute_scratch_bytes(int64_t R, int E);
+cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts,
+                           int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                           int32_t* scratch, int* status, cudaStream_t stream, int* launches);
+
+// Weighted top-k combine.
+cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* assign2row,
+                           uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,
+                           int* launches);
+
+// 1x128 e4m3 activation quantiser.
+cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, int64_t T, int H,
+                           cudaStream_t stream, int* launches);
+
+// MXFP4 weight preparation (K32 UE8M0 scales).
+cudaError_t launch_quant_w_mxfp4(const uint16_t* w, uint8_t* packed, uint8_t* sf, int64_t rows,
+                                 int K, cudaStream_t stream, int* launches);
+
+struct GemmProblem {
+  int64_t T;      // tokens (GEMM1 A rows)
+  int64_t R;      // routed rows
+  int H, I, E, k;
+  uint64_t wait_limit_ns;
+};
+
+// Grouped GEMM1 + SwiGLU, BF16 (x gathered by row2assign, act expert-sorted).
+cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int32_t* row2assign,
+                              const int32_t* offsets, const uint16_t* w13, uint16_t* act,
+                              int* status, cudaStream_t stream, int* launches);
+
+// Grouped GEMM2, BF16 (act expert-sorted, y expert-sorted).
+cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
+                              const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
+                              int* launches);
+
+int num_sms();
+
+// Test hook: when non-zero, CTA 0 of each grouped-GEMM launch skips its first stage fill.
+extern int g_inject_stall;
+
+}  // namespace moe

@@ -18,3 +18,11 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def moelib():
+    """The CUDA library (built here if missing; nvcc cross-compiles without a GPU)."""
+    from mixture_experts_routed_histogram_b200 import build, _capi
+    build.build()
+    return _capi

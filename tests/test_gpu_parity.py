@@ -1,0 +1,230 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Indices (routing ids, counts, offsets, row2assign, assign2row) must be bit-exact; floating
+point outputs must meet max|err| <= 2e-2 * max|ref| and cosine >= 0.9999.  Every output
+buffer carries a canary tail that must survive (out-of-bounds stores)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (COS_BF16, assert_close, canary_intact, dev, f64, gpu_permute, gpu_route,
+                      oracle_route, to_dev_i32, with_canary, workspace)
+from mixture_experts_routed_histogram_b200 import _capi as C
+from mixture_experts_routed_histogram_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+W = I.WORKLOADS
+
+# Small shapes that span several tiles and ragged tails on every GEMM edge.
+SMALL = {
+    "tiny": W["tiny"],
+    "odd_h384_i192": I.Workload("odd", 129, 384, 192, 4, 2),          # I % 128 = 64, H % 256 != 0
+    "one_token": I.Workload("one", 1, 256, 128, 8, 2),
+    "seven_tokens_e512_k10": I.Workload("e512", 7, 256, 128, 512, 10, routing="uniform"),
+    "sigmoid_top1": I.Workload("sig", 200, 512, 256, 16, 1, score="sigmoid", renorm=False),
+    "zipf_empty_experts": I.Workload("zipf", 96, 512, 384, 8, 2, routing="zipf"),
+    "many_tiles": I.Workload("many", 1000, 512, 256, 8, 4),
+}
+
+
+def _skewed_logits(wl, x):
+    lg = I.make_logits(wl, x)
+    lg[:, 3] += 100.0  # every token's top-1 is expert 3
+    return lg
+
+
+# ------------------------------------------------------------------ routing / permutation
+
+ROUTE_CASES = {
+    "tiny": W["tiny"],
+    "qwen3_30b_a3b": W["qwen3_30b_a3b"],
+    "llama4_scout": W["llama4_scout"],
+    "fp8_mxfp4_T16384": W["fp8_mxfp4"].with_T(16384),
+    "decode_T256": W["decode"].with_T(256),
+    "e1000_k32": I.Workload("wide", 300, 256, 128, 1000, 32),
+}
+
+
+@pytest.mark.parametrize("name", list(ROUTE_CASES))
+def test_route_and_permute_bitexact(name):
+    wl = ROUTE_CASES[name]
+    x = I.make_x(wl, 0, dev())
+    lg = I.make_logits(wl, x)
+    if name == "tiny":   # coarse logits: many exact ties
+        lg = torch.round(lg * 2) / 2
+    shape = C.MoeShape.from_workload(wl)
+    ids, w = gpu_route(shape, lg)
+    oids, ow = oracle_route(wl, lg)
+    assert np.array_equal(ids.cpu().numpy(), oids)
+    assert np.allclose(w.cpu().numpy(), ow, rtol=2e-6, atol=2e-7)
+    ws = workspace(shape)
+    # permutation of the oracle's ids (an input independent of the CUDA path)
+    counts, offsets, r2a, a2r = gpu_permute(shape, to_dev_i32(oids), ws)
+    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E)
+    assert np.array_equal(counts.cpu().numpy(), oc)
+    assert np.array_equal(offsets.cpu().numpy(), oo)
+    assert np.array_equal(r2a.cpu().numpy(), or2a)
+    assert np.array_equal(a2r.cpu().numpy(), oa2r)
+    assert C.moe_get_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("R,E", [(1, 1), (5, 8), (2048, 4), (2049, 300), (163840, 512),
+                                 (65536, 128), (600000, 64)])
+def test_permute_random_ids_bitexact(R, E):
+    rng = np.random.default_rng(R + E)
+    ids = rng.integers(0, E, R).astype(np.int32)
+    if E >= 8:
+        ids[rng.random(R) < 0.5] = 3             # heavy skew
+    shape = C.MoeShape.of(R, 64, 64, E, 1)
+    ws = workspace(shape)
+    counts, offsets, r2a, a2r = gpu_permute(shape, to_dev_i32(ids.reshape(R, 1)), ws)
+    oc, oo, or2a, oa2r = oracle.permute(ids.reshape(R, 1), E)
+    assert np.array_equal(counts.cpu().numpy(), oc)
+    assert np.array_equal(offsets.cpu().numpy(), oo)
+    assert np.array_equal(r2a.cpu().numpy(), or2a)
+    assert np.array_equal(a2r.cpu().numpy(), oa2r)
+
+
+def test_permute_flags_bad_ids():
+    shape = C.MoeShape.of(4, 64, 64, 8, 1)
+    ws = workspace(shape)
+    gpu_permute(shape, to_dev_i32(np.array([[0], [8], [1], [2]])), ws)
+    assert C.moe_get_device_status(ws) == C.MOE_ERR_DEVICE_BAD_INDEX
+    assert C.moe_get_device_status(ws) == 0  # read clears it
+
+
+# ------------------------------------------------------------------ GEMM stages
+
+def _stage_inputs(wl, skew=False):
+    inp = I.make_inputs(wl, 0, dev())
+    lg = _skewed_logits(wl, inp["x"]) if skew else inp["logits"]
+    oids, ow = oracle_route(wl, lg)
+    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E)
+    return inp, oids, ow, oo, or2a, oa2r
+
+
+GEMM_CASES = dict(SMALL)
+GEMM_CASES["skew_one_expert"] = I.Workload("skew", 300, 256, 128, 8, 1)
+
+
+@pytest.mark.parametrize("name", list(GEMM_CASES))
+def test_gemm1_swiglu_parity(name):
+    wl = GEMM_CASES[name]
+    inp, oids, ow, oo, or2a, oa2r = _stage_inputs(wl, skew=name.startswith("skew"))
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    R = wl.R
+    buf, act = with_canary(R, wl.I)
+    C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, to_dev_i32(or2a), to_dev_i32(oo),
+                               inp["w13"], None, act, None, ws)
+    torch.cuda.synchronize()
+    assert C.moe_get_device_status(ws) == 0
+    assert canary_intact(buf, R, wl.I)
+    tok = or2a.astype(np.int64) // wl.k
+    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), tok, ex)
+    assert_close(f64(act), ref, what=f"gemm1 {name}")
+
+
+@pytest.mark.parametrize("name", list(GEMM_CASES))
+def test_gemm2_parity(name):
+    wl = GEMM_CASES[name]
+    inp, oids, ow, oo, or2a, oa2r = _stage_inputs(wl, skew=name.startswith("skew"))
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    R = wl.R
+    g = torch.Generator(device=dev()).manual_seed(5)
+    act = torch.randn(R, wl.I, generator=g, device=dev()).to(torch.bfloat16)
+    buf, y = with_canary(R, wl.H)
+    C.moe_grouped_gemm2(shape, act, None, to_dev_i32(oo), inp["w2"], None, y, ws)
+    torch.cuda.synchronize()
+    assert C.moe_get_device_status(ws) == 0
+    assert canary_intact(buf, R, wl.H)
+    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    ref = oracle.gemm2_bf16_rows(I.bits(act), I.bits(inp["w2"]), np.arange(R), ex)
+    assert_close(f64(y), ref, what=f"gemm2 {name}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "odd_h384_i192", "seven_tokens_e512_k10"])
+def test_combine_parity(name):
+    wl = SMALL[name]
+    inp, oids, ow, oo, or2a, oa2r = _stage_inputs(wl)
+    shape = C.MoeShape.from_workload(wl)
+    g = torch.Generator(device=dev()).manual_seed(6)
+    y = torch.randn(wl.R, wl.H, generator=g, device=dev()).to(torch.bfloat16)
+    w32 = ow.astype(np.float32)
+    buf, out = with_canary(wl.T, wl.H)
+    C.moe_combine(shape, y, torch.from_numpy(w32).to(dev()), to_dev_i32(oa2r), out)
+    torch.cuda.synchronize()
+    assert canary_intact(buf, wl.T, wl.H)
+    ref, refb = oracle.combine(I.bits(y), w32, oa2r)
+    got = f64(out)
+    # one fp32 sum of k terms, one bf16 rounding: within one bf16 ulp of the oracle
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-30)
+
+
+# ------------------------------------------------------------------ whole forward pass
+
+def _forward(wl, inp, logits, ws):
+    shape = C.MoeShape.from_workload(wl)
+    buf, out = with_canary(wl.T, wl.H)
+    ids = torch.empty(wl.T, wl.k, dtype=torch.int32, device=dev())
+    C.moe_forward(shape, inp["x"], logits, inp["w13"], None, inp["w2"], None, out, ids, ws)
+    torch.cuda.synchronize()
+    assert canary_intact(buf, wl.T, wl.H)
+    return out, ids
+
+
+def _check_forward(wl, inp, logits, tokens, skew=False):
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    out, ids = _forward(wl, inp, logits, ws)
+    assert C.moe_get_device_status(ws) == 0
+    oids, ow = oracle_route(wl, logits)
+    assert np.array_equal(ids.cpu().numpy(), oids)
+    ref, _ = oracle.forward_bf16(I.bits(inp["x"]), oids, ow, I.bits(inp["w13"]),
+                                 I.bits(inp["w2"]), tokens)
+    got = f64(out)[tokens]
+    return assert_close(got, ref, COS_BF16, what=f"forward {wl.name} T={wl.T}"), (out, ws)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small_parity(name):
+    wl = SMALL[name]
+    inp = I.make_inputs(wl, 0, dev())
+    _check_forward(wl, inp, inp["logits"], np.arange(wl.T))
+
+
+def test_forward_skewed_one_expert():
+    wl = I.Workload("skew", 300, 256, 128, 8, 1)
+    inp = I.make_inputs(wl, 0, dev())
+    _check_forward(wl, inp, _skewed_logits(wl, inp["x"]), np.arange(wl.T))
+
+
+def test_forward_deterministic():
+    wl = SMALL["many_tiles"]
+    inp = I.make_inputs(wl, 0, dev())
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    a, _ = _forward(wl, inp, inp["logits"], ws)
+    b, _ = _forward(wl, inp, inp["logits"], ws)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+FULL = {
+    "qwen3_30b_a3b": W["qwen3_30b_a3b"],
+    "llama4_scout": W["llama4_scout"],
+    **{f"decode_T{t}": W["decode"].with_T(t) for t in I.DECODE_T_SWEEP},
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_forward_full_size_parity(name):
+    """Full-size workloads in the launch configuration the benchmark times; the oracle
+    checks a seeded token subset (always including the first and last token)."""
+    wl = FULL[name]
+    inp = I.make_inputs(wl, 0, dev())
+    n = 64 if wl.name == "decode" else 256
+    _check_forward(wl, inp, inp["logits"], I.parity_tokens(wl.T, n))

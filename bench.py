@@ -95,7 +95,8 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []       # (host arrival time, csv line)
+        self.window = None    # (t0, t1) of the timed region
 
     def __enter__(self):
         try:
@@ -105,13 +106,19 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0:   # first sample is in
+                time.sleep(0.01)
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -127,7 +134,13 @@ class ClockSampler:
             return None
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.window is not None:
+            inside = [ln for t, ln in lines if self.window[0] <= t <= self.window[1] + 0.15]
+            lines = inside if inside else [ln for _, ln in lines[-2:]]
+        else:
+            lines = [ln for _, ln in lines]
+        for ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -234,11 +247,13 @@ def bench_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        h0 = time.time()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.mark(h0, time.time())
     barrier(world)
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, world)
@@ -259,30 +274,53 @@ def bench_ours(args, rank, world, local):
     counts = bufs["counts"].cpu().numpy()
     flops_s, bytes_s, b_alg, ne = algorithmic(wl, counts)
 
-    # ---- end to end through the public API: pinned host input -> device -> host output
+    # ---- end to end through the public API: every step copies its inputs from pinned host
+    # memory and reads its output back; copies run on their own streams, double-buffered,
+    # so step i+1's upload and step i-1's download overlap step i's kernels.
     x_h = inp["x"].cpu().pin_memory()
     lg_h = inp["logits"].cpu().pin_memory()
-    out_h = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty_like(inp["x"])
-    lg_d = torch.empty_like(inp["logits"])
+    out_h = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_d = [torch.empty_like(inp["x"]) for _ in range(2)]
+    lg_d = [torch.empty_like(inp["logits"]) for _ in range(2)]
+    out_d = [torch.empty_like(out) for _ in range(2)]
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+    up_done = [torch.cuda.Event() for _ in range(2)]
+    fwd_done = [torch.cuda.Event() for _ in range(2)]
+    down_done = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        C.moe_forward(shape, x_d, lg_d, inp["w13"], None, inp["w2"], None, out, None, ws)
-        out_h.copy_(out, non_blocking=True)
+    def e2e_run(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(up_s):
+                if i >= 2:
+                    up_s.wait_event(fwd_done[b])          # inputs of step i-2 consumed
+                x_d[b].copy_(x_h, non_blocking=True)
+                lg_d[b].copy_(lg_h, non_blocking=True)
+                up_done[b].record(up_s)
+            stream.wait_event(up_done[b])
+            if i >= 2:
+                stream.wait_event(down_done[b])            # output buffer of step i-2 read
+            C.moe_forward(shape, x_d[b], lg_d[b], inp["w13"], None, inp["w2"], None, out_d[b],
+                          None, ws, stream)
+            fwd_done[b].record(stream)
+            with torch.cuda.stream(down_s):
+                down_s.wait_event(fwd_done[b])
+                out_h[b].copy_(out_d[b], non_blocking=True)
+                down_done[b].record(down_s)
+        stream.wait_stream(up_s)
+        stream.wait_stream(down_s)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    e2e_run(max(2, args.warmup))
     torch.cuda.synchronize()
     barrier(world)
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    up_s.wait_event(e2)
+    e2e_run(args.steps)
     e3.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e2.elapsed_time(e3) / args.steps, world)
+    assert torch.equal(out_h[(args.steps - 1) % 2].view(torch.int16), out.cpu().view(torch.int16))
 
     flops = wl.flops()
     tflops = flops * world / (ms_max * 1e-3) / 1e12
@@ -335,7 +373,8 @@ def bench_ours(args, rank, world, local):
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": x_h.numel() * 2 + lg_h.numel() * 4,
-                "d2h_bytes_per_step": out_h.numel() * 2},
+                "d2h_bytes_per_step": out_h[0].numel() * 2,
+                "pipelining": "H2D/D2H on separate streams, double-buffered across steps"},
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -428,7 +467,7 @@ def bench_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3_30b_a3b", choices=list(I.WORKLOADS))

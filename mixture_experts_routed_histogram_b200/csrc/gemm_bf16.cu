@@ -30,7 +30,10 @@
 // unwinds all roles, drains in-flight copies and MMAs and frees its TMEM.
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+
 #include <mutex>
+#include <string>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -40,11 +43,22 @@ namespace {
 
 constexpr int BM = 128;        // rows per tile (MMA M)
 constexpr int BK = 64;         // bf16 elements per 128-byte swizzled row
-constexpr int kThreads = 192;  // 6 warps
+
+// How the A operand reaches shared memory.
+enum AMode : int {
+  kATile = 0,     // contiguous rows: one 2-D TMA box per stage (GEMM2)
+  kAGather4 = 1,  // token rows: 32 TMA tile::gather4 loads per stage (GEMM1 alternative)
+  kACpAsync = 2,  // token rows: 4 loader warps, 16-byte cp.async into the swizzled layout
+};
+constexpr int kLoaderWarps = 4;
+__host__ __device__ constexpr int threads_for(int amode) {
+  return amode == kACpAsync ? 32 * (6 + kLoaderWarps) : 192;
+}
 
 struct KArgs {
   const int32_t* offsets;      // [E+1]
   const int32_t* row2assign;   // GEMM1 only
+  const uint16_t* a_rows;      // GEMM1 cp.async mode: x [T][K]
   uint16_t* out;               // act [R][I] (GEMM1) or y [R][H] (GEMM2)
   int* status;
   int E, k_top;
@@ -91,11 +105,13 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
 
-template <bool GEMM1, int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GEMM1, int AMODE, int BN, int STAGES>
+__global__ void __launch_bounds__(threads_for(AMODE), 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const KArgs args) {
   using L = Layout<BN, STAGES>;
+  constexpr int kThreads = threads_for(AMODE);
+  static_assert(GEMM1 || AMODE == kATile, "GEMM2 reads contiguous rows");
   constexpr int BN_OUT = GEMM1 ? BN / 2 : BN;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32<BM, BN>();
@@ -123,7 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = __ldg(args.offsets + i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // cp.async mode: the B producer's expect-tx arrival + one per loader thread
+      mbar_init(&full[s], AMODE == kACpAsync ? 1 + 32 * kLoaderWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = s_off[e] + mt * BM;
       const int rows = min(BM, s_off[e + 1] - row0);
       int tk0 = 0, tk1 = 0, tk2 = 0, tk3 = 0;
-      if constexpr (GEMM1) {
+      if constexpr (AMODE == kAGather4) {
         const int r = lane * 4;
         tk0 = __ldg(args.row2assign + row0 + (r + 0 < rows ? r + 0 : 0)) / args.k_top;
         tk1 = __ldg(args.row2assign + row0 + (r + 1 < rows ? r + 1 : 0)) / args.k_top;
@@ -207,10 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* a_dst = smem + s * L::STAGE;
         uint8_t* b_dst = a_dst + L::A_BYTES;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], L::STAGE);
+        if (lane == 0)
+          mbar_arrive_expect_tx(&full[s], AMODE == kACpAsync ? L::B_BYTES : L::STAGE);
         __syncwarp();
         if constexpr (GEMM1) {
-          tma_gather4(a_dst + lane * 4 * 128, &tmA, &full[s], kb * BK, tk0, tk1, tk2, tk3);
+          if constexpr (AMODE == kAGather4)
+            tma_gather4(a_dst + lane * 4 * 128, &tmA, &full[s], kb * BK, tk0, tk1, tk2, tk3);
           if (lane == 0) {
             tma_load_2d(b_dst, &tmB, &full[s], kb * BK, brow);
             tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[s], kb * BK, brow + args.n_out);
@@ -253,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if constexpr (AMODE == kACpAsync) fence_async_smem();  // cp.async data -> MMA reads
           tc_fence_after();
           const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + s * L::STAGE));
           const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + s * L::STAGE + L::A_BYTES));
@@ -275,6 +295,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ A gather (cp.async)
+    if constexpr (AMODE == kACpAsync) {
+      const int lw = warp - 6;
+      const int sub = lane >> 3;    // row within a group of 4
+      const int chunk = lane & 7;   // 16-byte chunk within the 128-byte row
+      uint32_t fill = 0;
+      bool ok = true;
+      for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
+        int e, mt, nt;
+        decode_task(task, s_tile, E, args.n_tiles, e, mt, nt);
+        const int row0 = s_off[e] + mt * BM;
+        const int rows = min(BM, s_off[e + 1] - row0);
+        const uint16_t* src[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = lw * 32 + i * 4 + sub;
+          const int tok = __ldg(args.row2assign + row0 + (r < rows ? r : 0)) / args.k_top;
+          src[i] = args.a_rows + static_cast<int64_t>(tok) * args.K + chunk * 8;
+        }
+        for (int kb = 0; kb < kblocks; ++kb, ++fill) {
+          const int s = fill % STAGES;
+          const uint32_t ph = (fill / STAGES) & 1u;
+          if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, s_abort, lim))) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_base = smem_u32(smem + s * L::STAGE);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = lw * 32 + i * 4 + sub;
+            cp_async_16(a_base + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * BK);
+          }
+          cp_async_mbar_arrive_noinc(&full[s]);
+        }
+      }
+      if (!ok && lane == 0) {
+        *s_abort = 1;
+        set_status(args.status, kStatusTimeout);
+      }
+      cp_async_wait_all();
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp can access
@@ -388,16 +450,26 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS;
 }
 
-template <bool GEMM1, int BN, int STAGES>
+template <bool GEMM1, int AMODE, int BN, int STAGES>
 cudaError_t run(const CUtensorMap& a, const CUtensorMap& b, const KArgs& args,
                 cudaStream_t stream) {
   using L = Layout<BN, STAGES>;
-  auto kern = grouped_gemm_bf16_kernel<GEMM1, BN, STAGES>;
+  auto kern = grouped_gemm_bf16_kernel<GEMM1, AMODE, BN, STAGES>;
   static cudaError_t attr = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (attr != cudaSuccess) return attr;
-  kern<<<num_sms(), kThreads, L::ALLOC, stream>>>(a, b, args);
+  kern<<<num_sms(), threads_for(AMODE), L::ALLOC, stream>>>(a, b, args);
   return cudaGetLastError();
+}
+
+// GEMM1 A-operand path: cp.async gather (default) or TMA gather4 (MOE_GEMM1_GATHER=tma4,
+// a tuning switch).
+bool use_gather4() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_GEMM1_GATHER");
+    return e && std::string(e) == "tma4";
+  }();
+  return v;
 }
 
 }  // namespace
@@ -427,6 +499,7 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   KArgs a{};
   a.offsets = offsets;
   a.row2assign = row2assign;
+  a.a_rows = x;
   a.out = act;
   a.status = status;
   a.E = p.E;
@@ -438,7 +511,11 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return wide ? run<true, 256, 4>(ta, tb, a, stream) : run<true, 128, 6>(ta, tb, a, stream);
+  if (use_gather4())
+    return wide ? run<true, kAGather4, 256, 4>(ta, tb, a, stream)
+                : run<true, kAGather4, 128, 6>(ta, tb, a, stream);
+  return wide ? run<true, kACpAsync, 256, 4>(ta, tb, a, stream)
+              : run<true, kACpAsync, 128, 6>(ta, tb, a, stream);
 }
 
 cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
@@ -463,7 +540,7 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run<false, bn, 4>(ta, tb, a, stream);
+  return run<false, kATile, bn, 4>(ta, tb, a, stream);
 }
 
 }  // namespace moe

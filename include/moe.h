@@ -109,6 +109,27 @@ MOE_API moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, i
                          int32_t *offsets, int32_t *row2assign, int32_t *assign2row, void *ws,
                          size_t ws_bytes, cudaStream_t stream);
 
+/* Allocation-free variant of moe_permute, for callers that cannot hand the library a
+ * workspace: host code that runs where device allocation is not allowed or not
+ * possible -- for example an integration layer whose memory is a fixed pool reserved at
+ * start-up and which has no scratch buffer to pass down.  (This entry point has no
+ * counterpart on the pages; it is a packaging variant of the permutation above.)
+ * Same inputs, outputs and results as moe_permute, bit for bit.  The per-chunk
+ * histograms live in a 256 KB file-scope device array instead of the workspace; it
+ * needs ceil(T*k / chunk) * E <= 65536, where chunk = 2048 while T*k <= 524288 (so
+ * E = 512 works up to T*k = 262144 and E = 128 up to 524288; beyond 524288 the chunk
+ * grows so that there are 256 chunks, which needs E <= 256).  Larger problems return
+ * MOE_ERR_UNSUPPORTED_SHAPE without launching anything.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture.  Every call shares the array: calls
+ * whose kernels overlap on the GPU (other streams, other host threads) race on it;
+ * calls ordered on one stream are safe, and no state carries over between them.  Ids
+ * outside [0, E) are skipped, as in moe_permute, but there is no status word to record
+ * them in.  Calls no cudaMalloc, cudaFree or allocating library routine. */
+MOE_API moe_status_t moe_permute_noalloc(const moe_shape_t *shape, const int32_t *ids,
+                                         int32_t *counts, int32_t *offsets, int32_t *row2assign,
+                                         int32_t *assign2row, cudaStream_t stream);
+
 /* Block-scaled path: per token and per 128 consecutive columns, the smallest power of two
  * s = 2^e (e clamped to [-127,127]) with max|x| <= 448*s, and e4m3 codes of x/s (round to
  * nearest even, saturating).  TileScale PR #70 "Design" (FP8 E4M3, fp32 per-128 scales).

@@ -34,7 +34,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute
            "moe_quantize_x", "moe_quantize_weights_mxfp4", "moe_grouped_gemm1_swiglu",
            "moe_grouped_gemm2", "moe_combine", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_debug_set_wait_limit_ns", "moe_debug_inject_stall",
-           "moe_last_launch_count")
+           "moe_last_launch_count", "moe_permute_noalloc")
 
 
 class MoeShape(ctypes.Structure):
@@ -78,6 +78,8 @@ def load():
             L.moe_workspace_init.argtypes = [vp, sz, vp]; L.moe_workspace_init.restype = st
             L.moe_route.argtypes = [S, vp, vp, vp, vp]; L.moe_route.restype = st
             L.moe_permute.argtypes = [S, vp, vp, vp, vp, vp, vp, sz, vp]; L.moe_permute.restype = st
+            L.moe_permute_noalloc.argtypes = [S, vp, vp, vp, vp, vp, vp]
+            L.moe_permute_noalloc.restype = st
             L.moe_quantize_x.argtypes = [S, vp, vp, vp, vp]; L.moe_quantize_x.restype = st
             L.moe_quantize_weights_mxfp4.argtypes = [ctypes.c_int64, ctypes.c_int32, vp, vp, vp, vp]
             L.moe_quantize_weights_mxfp4.restype = st
@@ -150,6 +152,13 @@ def moe_permute(shape, ids, counts, offsets, row2assign, assign2row, ws, stream=
     _check(load().moe_permute(ctypes.byref(shape), _p(ids), _p(counts), _p(offsets),
                               _p(row2assign), _p(assign2row), _p(ws), _nbytes(ws), _s(stream)),
            "moe_permute")
+
+
+def moe_permute_noalloc(shape, ids, counts, offsets, row2assign, assign2row, stream=None):
+    """moe_permute without a workspace (its scratch is a static device array)."""
+    _check(load().moe_permute_noalloc(ctypes.byref(shape), _p(ids), _p(counts), _p(offsets),
+                                      _p(row2assign), _p(assign2row), _s(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_quantize_x(shape, x, xq, sx, stream=None):

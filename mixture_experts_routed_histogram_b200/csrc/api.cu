@@ -146,6 +146,22 @@ moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* ids, int32_t* 
   return cuda_status(e);
 }
 
+moe_status_t moe_permute_noalloc(const moe_shape_t* shape, const int32_t* ids, int32_t* counts,
+                                 int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                 cudaStream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_shape(shape));
+  MOE_TRY(need_ptrs({counts, offsets}));
+  const int64_t R = shape->T * shape->k;
+  if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
+  if (!moe::permute_noalloc_fits(R, shape->E)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  int n = 0;
+  cudaError_t e = moe::launch_permute_noalloc(ids, R, shape->E, counts, offsets, row2assign,
+                                              assign2row, stream, &n);
+  g_last_launches = n;
+  return cuda_status(e);
+}
+
 moe_status_t moe_quantize_x(const moe_shape_t* shape, const uint16_t* x, uint8_t* xq, float* sx,
                             cudaStream_t stream) {
   g_last_launches = 0;

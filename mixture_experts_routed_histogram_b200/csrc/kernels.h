@@ -22,6 +22,13 @@ cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts
                            int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                            int32_t* scratch, int* status, cudaStream_t stream, int* launches);
 
+// The same permutation with its per-chunk histograms in a static device array (no
+// workspace); fits() tells whether ceil(R / chunk) * E stays within that array.
+bool permute_noalloc_fits(int64_t R, int E);
+cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t R, int E, int32_t* counts,
+                                   int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                   cudaStream_t stream, int* launches);
+
 // Weighted top-k combine.
 cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* assign2row,
                            uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,

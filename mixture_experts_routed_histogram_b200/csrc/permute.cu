@@ -16,6 +16,8 @@
 //      ranking equal experts inside a warp with __match_any_sync and across the 8 warps
 //      with round-stamped per-warp counts, so the row of assignment a is offsets[e] +
 //      #{a' < a : ids[a'] == e}: the stable order.
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -186,6 +188,70 @@ cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts
   const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
   *launches += 2;
   chunk_hist_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, scratch, status);
+  scatter_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, nchunks, scratch, counts,
+                                                   offsets, row2assign, assign2row);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// For callers that cannot hand the library a workspace: the per-chunk histograms live in
+// this file-scope device array instead (256 KB, held on every device that loads the
+// library until the process exits).  Every call shares it, so two calls whose kernels
+// overlap on the GPU (different streams, or different host threads) race on it; calls
+// serialised on one stream are safe.  The histogram kernel overwrites every entry a call
+// reads, so nothing has to be cleared between calls.
+
+constexpr int kNoAllocScratchInts = 1 << 16;
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device (with
+// that device current) and cached.
+static cudaError_t noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+bool permute_noalloc_fits(int64_t R, int E) {
+  if (R == 0) return true;
+  const int64_t c = chunk_size(R);
+  const int64_t n = (R + c - 1) / c;
+  return n * E <= kNoAllocScratchInts;
+}
+
+cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t R, int E, int32_t* counts,
+                                   int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                   cudaStream_t stream, int* launches) {
+  if (R == 0) {
+    ++*launches;
+    cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
+    return cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
+  }
+  int32_t* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  const int chunk = chunk_size(R);
+  const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
+  *launches += 2;
+  chunk_hist_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, scratch, nullptr);
   scatter_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, nchunks, scratch, counts,
                                                    offsets, row2assign, assign2row);
   return cudaGetLastError();

@@ -168,40 +168,60 @@ def build_device_inputs(wl, seed):
 def run_stages(shape, wl, inp, ws, bufs, events=None):
     """One forward pass as separate C-ABI stage calls (same kernels as moe_forward),
     optionally bracketing each stage with CUDA events for the per-kernel breakdown."""
-    def mark(i):
+    fp8 = wl.dtype == "fp8_mxfp4"
+    marks = iter(range(len(stages_of(wl)) + 1))
+
+    def mark():
+        i = next(marks)
         if events is not None:
             events[i].record()
-    mark(0)
+    mark()
     C.moe_route(shape, inp["logits"], bufs["ids"], bufs["w"])
-    mark(1)
+    mark()
     C.moe_permute(shape, bufs["ids"], bufs["counts"], bufs["offsets"], bufs["r2a"], bufs["a2r"], ws)
-    mark(2)
-    C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, bufs["r2a"], bufs["offsets"], inp["w13"],
-                               None, bufs["act"], None, ws)
-    mark(3)
-    C.moe_grouped_gemm2(shape, bufs["act"], None, bufs["offsets"], inp["w2"], None, bufs["y"], ws)
-    mark(4)
+    mark()
+    if fp8:
+        C.moe_quantize_x(shape, inp["x"], bufs["xq"], bufs["sx"])
+        mark()
+        C.moe_grouped_gemm1_swiglu(shape, bufs["xq"], bufs["sx"], bufs["r2a"], bufs["offsets"],
+                                   inp["w13"], inp["w13_sf"], bufs["act"], bufs["act_sf"], ws)
+        mark()
+        C.moe_grouped_gemm2(shape, bufs["act"], bufs["act_sf"], bufs["offsets"], inp["w2"],
+                            inp["w2_sf"], bufs["y"], ws)
+    else:
+        C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, bufs["r2a"], bufs["offsets"], inp["w13"],
+                                   None, bufs["act"], None, ws)
+        mark()
+        C.moe_grouped_gemm2(shape, bufs["act"], None, bufs["offsets"], inp["w2"], None, bufs["y"], ws)
+    mark()
     C.moe_combine(shape, bufs["y"], bufs["w"], bufs["a2r"], bufs["out"])
-    mark(5)
+    mark()
 
 
-STAGES = ["route", "permute", "gemm1_swiglu", "gemm2", "combine"]
+def stages_of(wl):
+    if wl.dtype == "fp8_mxfp4":
+        return ["route", "permute", "quantize_x", "gemm1_swiglu", "gemm2", "combine"]
+    return ["route", "permute", "gemm1_swiglu", "gemm2", "combine"]
 
 
 def algorithmic(wl, counts):
     """Algorithmic FLOPs and bytes of each stage for the actual per-expert counts."""
     T, H, Ii, E, k, R = wl.T, wl.H, wl.I, wl.E, wl.k, wl.R
     ne = int((counts > 0).sum())
+    fp8 = wl.dtype == "fp8_mxfp4"
+    wbytes = (0.5 + 1.0 / 32) if fp8 else 2.0     # per weight element (codes + scales)
+    abytes = (1.0 + 4.0 / 128) if fp8 else 2.0     # per activation element (codes + scales)
     f = {"gemm1_swiglu": 4.0 * R * H * Ii, "gemm2": 2.0 * R * H * Ii}
     b = {
         "route": T * E * 4 + R * 8,
         "permute": R * 4 * 3 + E * 8,
-        "gemm1_swiglu": ne * 2 * Ii * H * 2 + T * H * 2 + R * Ii * 2 + R * 4,
-        "gemm2": ne * H * Ii * 2 + R * Ii * 2 + R * H * 2,
+        "quantize_x": T * H * 2 + T * H * abytes,
+        "gemm1_swiglu": ne * 2 * Ii * H * wbytes + T * H * abytes + R * Ii * abytes + R * 4,
+        "gemm2": ne * H * Ii * wbytes + R * Ii * abytes + R * H * 2,
         "combine": R * H * 2 + T * H * 2 + R * 8,
     }
     # whole-pass bytes without the y round trip (a fused combine could avoid it)
-    b_alg = (ne * 3 * Ii * H * 2 + T * H * 2 * 2 + R * Ii * 2 * 2 + T * E * 4 + R * 16)
+    b_alg = (ne * 3 * Ii * H * wbytes + T * H * 2 * 2 + R * Ii * abytes * 2 + T * E * 4 + R * 16)
     return f, b, b_alg, ne
 
 
@@ -230,11 +250,16 @@ def bench_ours(args, rank, world, local):
         "y": torch.empty(R, wl.H, dtype=torch.bfloat16, device="cuda"),
         "out": out,
     }
+    if wl.dtype == "fp8_mxfp4":
+        bufs["act"] = torch.empty(R, wl.I, dtype=torch.uint8, device="cuda")
+        bufs["act_sf"] = torch.empty(R, wl.I // 128, dtype=torch.float32, device="cuda")
+        bufs["xq"] = torch.empty(wl.T, wl.H, dtype=torch.uint8, device="cuda")
+        bufs["sx"] = torch.empty(wl.T, wl.H // 128, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
-        C.moe_forward(shape, inp["x"], inp["logits"], inp["w13"], None, inp["w2"], None, out,
-                      None, ws)
+        C.moe_forward(shape, inp["x"], inp["logits"], inp["w13"], inp["w13_sf"], inp["w2"],
+                      inp["w2_sf"], out, None, ws)
 
     # warm-up
     for _ in range(args.warmup):
@@ -264,6 +289,7 @@ def bench_ours(args, rank, world, local):
     # ---- per-kernel breakdown (stage calls, events on the launching stream)
     run_stages(shape, wl, inp, ws, bufs)
     torch.cuda.synchronize()
+    STAGES = stages_of(wl)
     acc = np.zeros(len(STAGES))
     for _ in range(args.steps):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
@@ -300,8 +326,8 @@ def bench_ours(args, rank, world, local):
             stream.wait_event(up_done[b])
             if i >= 2:
                 stream.wait_event(down_done[b])            # output buffer of step i-2 read
-            C.moe_forward(shape, x_d[b], lg_d[b], inp["w13"], None, inp["w2"], None, out_d[b],
-                          None, ws, stream)
+            C.moe_forward(shape, x_d[b], lg_d[b], inp["w13"], inp["w13_sf"], inp["w2"],
+                          inp["w2_sf"], out_d[b], None, ws, stream)
             fwd_done[b].record(stream)
             with torch.cuda.stream(down_s):
                 down_s.wait_event(fwd_done[b])
@@ -325,25 +351,29 @@ def bench_ours(args, rank, world, local):
     flops = wl.flops()
     tflops = flops * world / (ms_max * 1e-3) / 1e12
     pk, pk_kind = peaks()
+    fp8 = wl.dtype == "fp8_mxfp4"
+    # FP8 x FP4 block-scaled MMA: the measured bf16 peak x the nominal 4.5/2.25 ratio
+    t_peak = pk["bf16_tflops"] * (2.0 if fp8 else 1.0)
     # dominant kernel: the stage with the largest measured share
     dom = int(np.argmax(stage_ms))
     dname = STAGES[dom]
     t_ker = stage_ms[dom] * 1e-3
     if dname in flops_s:
-        t_tensor = flops_s[dname] / (pk["bf16_tflops"] * 1e12)
+        t_tensor = flops_s[dname] / (t_peak * 1e12)
         t_hbm = bytes_s[dname] / (pk["hbm_gbs"] * 1e9)
     else:
         t_tensor, t_hbm = 0.0, 1.0
     if t_tensor >= t_hbm:
         roof = {"bound": "tensor", "achieved": flops_s[dname] / t_ker / 1e12,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+                "peak": t_peak, "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": bytes_s[dname] / t_ker / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
     roof["kernel"] = dname
-    roof["peak_source"] = f"{pk_kind} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["peak_source"] = (f"{pk_kind} " + ("copy" if roof["bound"] == "hbm" else
+                           ("burst bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 else "burst bf16")))
 
     result = {
         "metric": METRIC,
@@ -358,17 +388,17 @@ def bench_ours(args, rank, world, local):
         "scaling": "weak",
         "vs_baseline": (round(tflops / world / PUBLISHED[wl.name], 4)
                         if wl.name in PUBLISHED and wl.T == 8192 else None),
-        "dtype": "bf16",
+        "dtype": "e4m3 x e2m1 (fp32 accumulate)" if fp8 else "bf16",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, random-init)",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                    "score": wl.score, "routing": wl.routing, "parallelism": f"replicas x{world}",
                    "nonempty_experts": ne,
                    "l2": "inputs larger than L2 (weights %.2f GB re-read every step)" %
-                         ((3 * wl.E * wl.I * wl.H * 2) / 1e9)},
+                         ((3 * wl.E * wl.I * wl.H * ((0.5 + 1 / 32) if fp8 else 2)) / 1e9)},
         "hbm_gbs_alg": round(b_alg / (ms_max * 1e-3) / 1e9, 1),
         "hbm_frac_alg": round(b_alg / (ms_max * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "roofline": roof,
-        "stages_ms": {s: round(float(v), 4) for s, v in zip(STAGES, stage_ms)},
+        "stages_ms": {st: round(float(v), 4) for st, v in zip(STAGES, stage_ms)},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4),
@@ -384,6 +414,20 @@ def bench_ours(args, rank, world, local):
 
 # ---------------------------------------------------------------- CPU oracle (baseline only)
 
+def _oracle_weights(wl, inp):
+    """Host copies of the weights in the form the oracle takes."""
+    if wl.dtype == "fp8_mxfp4":
+        return tuple(inp[k].cpu().numpy() for k in ("w13", "w13_sf", "w2", "w2_sf"))
+    return (I.bits(inp["w13"]), I.bits(inp["w2"]))
+
+
+def _oracle_forward(wl, x, ids, w, wts, toks):
+    import oracle
+    if wl.dtype == "fp8_mxfp4":
+        return oracle.forward_fp8_mxfp4(x, ids, w, *wts, tokens=toks, requant_act=True)
+    return oracle.forward_bf16(x, ids, w, wts[0], wts[1], toks)
+
+
 def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
     """Time the fp64 oracle on a bounded sample of the same workload: routing + permutation
     on all T tokens, the expert MLP on a token subset sized for the budget; TFLOP/s over
@@ -391,8 +435,7 @@ def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
     import oracle
     x = I.bits(inp["x"])
     lg = inp["logits"].cpu().numpy()
-    w13 = I.bits(inp["w13"])
-    w2 = I.bits(inp["w2"])
+    wts = _oracle_weights(wl, inp)
     score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
     t0 = time.perf_counter()
     ids, w = oracle.route(lg, wl.k, score, wl.renorm)
@@ -401,12 +444,12 @@ def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
     # probe the per-token cost on a few tokens, then size the sample for the budget
     probe = I.parity_tokens(wl.T, 4, seed=1)
     t0 = time.perf_counter()
-    oracle.forward_bf16(x, ids, w, w13, w2, probe)
+    _oracle_forward(wl, x, ids, w, wts, probe)
     per_tok = (time.perf_counter() - t0) / len(probe)
     n = int(max(4, min(wl.T, (budget_s - t_route) / max(per_tok, 1e-6)))) if T_sample is None else T_sample
     toks = I.parity_tokens(wl.T, n, seed=2)
     t0 = time.perf_counter()
-    oracle.forward_bf16(x, ids, w, w13, w2, toks)
+    _oracle_forward(wl, x, ids, w, wts, toks)
     t_mlp = time.perf_counter() - t0
     # scale the subset time to all T tokens; routing/permutation counted once
     t_full = t_route + t_mlp * wl.T / len(toks)
@@ -430,13 +473,12 @@ def bench_reference(args, rank, world):
     import oracle
     x = I.bits(inp["x"])
     lg = inp["logits"].cpu().numpy()
-    w13 = I.bits(inp["w13"])
-    w2 = I.bits(inp["w2"])
+    wts = _oracle_weights(wl, inp)
     score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
     ids, w = oracle.route(lg, wl.k, score, wl.renorm)
     probe = I.parity_tokens(wl.T, 4, seed=1)
     t0 = time.perf_counter()
-    oracle.forward_bf16(x, ids, w, w13, w2, probe)
+    _oracle_forward(wl, x, ids, w, wts, probe)
     per_tok = (time.perf_counter() - t0) / len(probe)
     per_step_budget = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     n = int(max(2, min(wl.T, per_step_budget / max(per_tok, 1e-6))))
@@ -445,7 +487,7 @@ def bench_reference(args, rank, world):
         toks = I.parity_tokens(wl.T, n, seed=10 + s)
         t0 = time.perf_counter()
         oracle.route(lg, wl.k, score, wl.renorm)
-        oracle.forward_bf16(x, ids, w, w13, w2, toks)
+        _oracle_forward(wl, x, ids, w, wts, toks)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)

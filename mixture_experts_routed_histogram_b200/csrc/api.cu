@@ -18,10 +18,12 @@ constexpr size_t kStatusBytes = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // Workspace regions (byte offsets from the workspace base).
 struct WsLayout {
-  size_t status, ids, w, counts, offsets, r2a, a2r, scratch, xq, sx, act, act_sf, y, total;
+  size_t status, ids, w, counts, offsets, r2a, a2r, scratch, xq, sx, sxw, act, act_sf, act_sfw,
+      y, total;
 };
 
 WsLayout layout(const moe_shape_t& s) {
@@ -39,8 +41,10 @@ WsLayout layout(const moe_shape_t& s) {
   L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(R), s.E));
   L.xq = o; o = up(o + (fp8 ? T * H : 0));
   L.sx = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
+  L.sxw = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
   L.act = o; o = up(o + (fp8 ? R * I : 2 * R * I));
   L.act_sf = o; o = up(o + (fp8 ? 4 * R * (I / 128) : 0));
+  L.act_sfw = o; o = up(o + (fp8 ? 4 * R * (I / 128) : 0));
   L.y = o; o = up(o + 2 * R * H);
   L.total = o;
   return L;
@@ -170,7 +174,7 @@ moe_status_t moe_quantize_x(const moe_shape_t* shape, const uint16_t* x, uint8_t
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({x, xq, sx}));
   int n = 0;
-  cudaError_t e = moe::launch_quant_x(x, xq, sx, shape->T, shape->H, stream, &n);
+  cudaError_t e = moe::launch_quant_x(x, xq, sx, nullptr, shape->T, shape->H, stream, &n);
   g_last_launches = n;
   return cuda_status(e);
 }
@@ -195,14 +199,27 @@ moe_status_t moe_grouped_gemm1_swiglu(const moe_shape_t* shape, const void* a, c
                                       float* act_sf, void* ws, size_t ws_bytes,
                                       cudaStream_t stream) {
   g_last_launches = 0;
-  (void)sa; (void)w13_sf; (void)act_sf;
   MOE_TRY(check_shape(shape));
-  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
   MOE_TRY(need_ptrs({offsets, ws}));
   if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({a, row2assign, w13, act}));
   int n = 0;
+  if (shape->dtype == MOE_DTYPE_FP8_MXFP4) {
+    MOE_TRY(need_ptrs({sa, w13_sf, act_sf}));
+    if (!aligned32(w13)) return MOE_ERR_MISALIGNED;
+    const WsLayout L = layout(*shape);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    uint32_t* sxw = at<uint32_t>(ws, L.sxw);
+    cudaError_t e = moe::launch_scale_words(sa, sxw, shape->T * (shape->H / 128), stream, &n);
+    if (e == cudaSuccess)
+      e = moe::launch_gemm1_mx(problem(*shape), static_cast<const uint8_t*>(a), sxw, row2assign,
+                               offsets, static_cast<const uint8_t*>(w13), w13_sf,
+                               static_cast<uint8_t*>(act), act_sf, at<uint32_t>(ws, L.act_sfw),
+                               status_word(ws), stream, &n);
+    g_last_launches = n;
+    return cuda_status(e);
+  }
   cudaError_t e = moe::launch_gemm1_bf16(problem(*shape), static_cast<const uint16_t*>(a),
                                          row2assign, offsets, static_cast<const uint16_t*>(w13),
                                          static_cast<uint16_t*>(act), status_word(ws), stream, &n);
@@ -214,14 +231,27 @@ moe_status_t moe_grouped_gemm2(const moe_shape_t* shape, const void* act, const 
                                const int32_t* offsets, const void* w2, const uint8_t* w2_sf,
                                uint16_t* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
   g_last_launches = 0;
-  (void)act_sf; (void)w2_sf;
   MOE_TRY(check_shape(shape));
-  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
   MOE_TRY(need_ptrs({offsets, ws}));
   if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({act, w2, y}));
   int n = 0;
+  if (shape->dtype == MOE_DTYPE_FP8_MXFP4) {
+    MOE_TRY(need_ptrs({act_sf, w2_sf}));
+    if (!aligned32(w2)) return MOE_ERR_MISALIGNED;
+    const WsLayout L = layout(*shape);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    uint32_t* asw = at<uint32_t>(ws, L.act_sfw);
+    const int64_t R = shape->T * shape->k;
+    cudaError_t e = moe::launch_scale_words(act_sf, asw, R * (shape->I / 128), stream, &n);
+    if (e == cudaSuccess)
+      e = moe::launch_gemm2_mx(problem(*shape), static_cast<const uint8_t*>(act), asw, offsets,
+                               static_cast<const uint8_t*>(w2), w2_sf, y, status_word(ws), stream,
+                               &n);
+    g_last_launches = n;
+    return cuda_status(e);
+  }
   cudaError_t e = moe::launch_gemm2_bf16(problem(*shape), static_cast<const uint16_t*>(act),
                                          offsets, static_cast<const uint16_t*>(w2), y,
                                          status_word(ws), stream, &n);
@@ -247,9 +277,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
                          const uint8_t* w2_sf, uint16_t* out, int32_t* ids_out, void* ws,
                          size_t ws_bytes, cudaStream_t stream) {
   g_last_launches = 0;
-  (void)w13_sf; (void)w2_sf;
   MOE_TRY(check_shape(shape));
-  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!ws) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_MISALIGNED;
   const WsLayout L = layout(*shape);
@@ -257,6 +285,11 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({x, logits, w13, w2, out}));
   if (ids_out && !aligned16(ids_out)) return MOE_ERR_MISALIGNED;
+  const bool fp8 = shape->dtype == MOE_DTYPE_FP8_MXFP4;
+  if (fp8) {
+    MOE_TRY(need_ptrs({w13_sf, w2_sf}));
+    if (!aligned32(w13) || !aligned32(w2)) return MOE_ERR_MISALIGNED;
+  }
 
   const int64_t T = shape->T, R = T * shape->k;
   int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
@@ -277,12 +310,28 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
   if ((e = moe::launch_permute(ids, R, shape->E, counts, offsets, r2a, a2r,
                                at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if ((e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+  if (fp8) {
+    uint8_t* xq = at<uint8_t>(ws, L.xq);
+    uint32_t* sxw = at<uint32_t>(ws, L.sxw);
+    uint8_t* aq = at<uint8_t>(ws, L.act);
+    uint32_t* asw = at<uint32_t>(ws, L.act_sfw);
+    if ((e = moe::launch_quant_x(x, xq, at<float>(ws, L.sx), sxw, T, shape->H, stream, &n)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((e = moe::launch_gemm1_mx(p, xq, sxw, r2a, offsets, static_cast<const uint8_t*>(w13),
+                                  w13_sf, aq, nullptr, asw, status, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((e = moe::launch_gemm2_mx(p, aq, asw, offsets, static_cast<const uint8_t*>(w2), w2_sf, y,
                                   status, stream, &n)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if ((e = moe::launch_gemm2_bf16(p, act, offsets, static_cast<const uint16_t*>(w2), y, status,
-                                  stream, &n)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+      return MOE_ERR_CUDA;
+  } else {
+    if ((e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+                                    status, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((e = moe::launch_gemm2_bf16(p, act, offsets, static_cast<const uint16_t*>(w2), y, status,
+                                    stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if ((e = moe::launch_combine(y, w, a2r, out, T, shape->H, shape->k, stream, &n)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 // One warp per (token, 128-column group); each lane owns 4 consecutive columns.
 __global__ void __launch_bounds__(256)
     quant_x_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ xq,
-                   float* __restrict__ sx, int64_t groups, int H) {
+                   float* __restrict__ sx, uint32_t* __restrict__ sxw, int64_t groups, int H) {
   const int lane = threadIdx.x & 31;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (gid >= groups) return;
@@ -79,7 +79,10 @@ __global__ void __launch_bounds__(256)
   const uint32_t lo = cvt_e4m3x2(f0 * inv, f1 * inv);
   const uint32_t hi = cvt_e4m3x2(f2 * inv, f3 * inv);
   *reinterpret_cast<uint32_t*>(xq + base) = lo | (hi << 16);
-  if (lane == 0) sx[t * G + g] = pow2f(s);
+  if (lane == 0) {
+    sx[t * G + g] = pow2f(s);
+    if (sxw) sxw[t * G + g] = static_cast<uint32_t>(s + 127) * 0x01010101u;
+  }
 }
 
 // One thread per (row, 32-element group).
@@ -140,12 +143,13 @@ cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* ass
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, int64_t T, int H,
-                           cudaStream_t stream, int* launches) {
+cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* sxw, int64_t T,
+                           int H, cudaStream_t stream, int* launches) {
   const int64_t groups = T * (H / 128);
   if (groups == 0) return cudaSuccess;
   ++*launches;
-  quant_x_kernel<<<static_cast<unsigned>((groups + 7) / 8), 256, 0, stream>>>(x, xq, sx, groups, H);
+  quant_x_kernel<<<static_cast<unsigned>((groups + 7) / 8), 256, 0, stream>>>(x, xq, sx, sxw,
+                                                                            groups, H);
   return cudaGetLastError();
 }
 

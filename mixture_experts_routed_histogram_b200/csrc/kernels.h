@@ -34,9 +34,14 @@ cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* ass
                            uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,
                            int* launches);
 
-// 1x128 e4m3 activation quantiser.
-cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, int64_t T, int H,
-                           cudaStream_t stream, int* launches);
+// 1x128 e4m3 activation quantiser; sxw (nullable) also receives the UE8M0 word of each
+// scale (its byte repeated four times), the form the block-scaled GEMMs read.
+cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* sxw, int64_t T,
+                           int H, cudaStream_t stream, int* launches);
+
+// fp32 power-of-two scales -> UE8M0 words.
+cudaError_t launch_scale_words(const float* s, uint32_t* w, int64_t n, cudaStream_t stream,
+                               int* launches);
 
 // MXFP4 weight preparation (K32 UE8M0 scales).
 cudaError_t launch_quant_w_mxfp4(const uint16_t* w, uint8_t* packed, uint8_t* sf, int64_t rows,
@@ -58,6 +63,18 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
 cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
                               const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
                               int* launches);
+
+// Block-scaled grouped GEMM1 + SwiGLU + 1x128 requantisation (e4m3 x MXFP4).
+cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint32_t* sxw,
+                            const int32_t* row2assign, const int32_t* offsets,
+                            const uint8_t* w13p, const uint8_t* w13sf, uint8_t* act,
+                            float* act_sf, uint32_t* act_sfw, int* status, cudaStream_t stream,
+                            int* launches);
+
+// Block-scaled grouped GEMM2 (e4m3 act x MXFP4 W2, bf16 y).
+cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint32_t* act_sfw,
+                            const int32_t* offsets, const uint8_t* w2p, const uint8_t* w2sf,
+                            uint16_t* y, int* status, cudaStream_t stream, int* launches);
 
 int num_sms();
 

@@ -125,6 +125,11 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
                : "memory");
 }
 
+// 4-byte global -> shared copy (cp.async.ca: 4 and 8 byte copies are allowed there).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
@@ -164,6 +169,54 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Block-scaled MMA: D[tmem] (+)= (A * 2^sfa) * (B * 2^sfb)^T with A e4m3 and B e2m1 in
+// shared memory, one UE8M0 scale per 32 K per row of A and of B read from TMEM.  The
+// scale byte inside each 32-bit TMEM word is chosen by the instruction descriptor's
+// sf-id fields (and the top two bits of the scale addresses).
+__device__ __forceinline__ void mma_mxf8f6f4_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t sfa_tmem,
+                                                uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem),
+      "r"(accumulate)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory (descriptor) into TMEM lanes 0-31, columns
+// taddr..taddr+3, broadcast to all four 32-lane quadrants.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Descriptor of 32 consecutive 16-byte shared-memory rows (no swizzle; 8-row core
+// matrices 128 bytes apart) -- the source layout of tmem_cp_32x128b_warpx4.
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address
+  d |= static_cast<uint64_t>(128u >> 4) << 32;         // stride byte offset: 8 rows x 16 B
+  d |= static_cast<uint64_t>(1u) << 46;                // descriptor version for sm_100
+  return d;                                            // swizzle mode 0: none
+}
+
+// Instruction descriptor for kind::mxf8f6f4.block_scale: A e4m3, B e2m1, UE8M0 scales
+// (one per 32 K), fp32 D, both K-major; k_sub selects the scale byte of A and B.
+template <int M, int N>
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_e2m1(uint32_t k_sub) {
+  static_assert(M == 128, "M");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N");
+  return (k_sub << 4)                                // B scale-factor id
+         | (0u << 7)                                 // A format: e4m3
+         | (5u << 10)                                // B format: e2m1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (1u << 23)                                // scale format: UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)     // M / 16
+         | (k_sub << 29);                            // A scale-factor id
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far completes.

@@ -98,6 +98,39 @@ def make_weights(wl: Workload, seed: int = 0, device="cpu"):
     return w13, w2
 
 
+# Synthetic MXFP4 weights are drawn directly as codes and scale bytes (no quantiser runs
+# here): magnitudes of the e2m1 codes 0..7 (values 0, .5, 1, 1.5, 2, 3, 4, 6) follow this
+# table, the sign is a fair coin, and each 32-element block's UE8M0 byte is
+# 127 + floor(log2(1/sqrt(fan_in))) - 2 + U{0,1,2}, so values have about the spread of
+# N(0, 1/fan_in) weights.
+E2M1_MAGNITUDE_PROBS = (0.16, 0.30, 0.20, 0.13, 0.10, 0.07, 0.03, 0.01)
+
+
+def _mx_block(rows: int, K: int, fan_in: int, g: torch.Generator, device):
+    probs = torch.tensor(E2M1_MAGNITUDE_PROBS, device=device)
+    mag = torch.multinomial(probs, rows * K, replacement=True, generator=g).to(torch.uint8)
+    sign = torch.randint(0, 2, (rows * K,), generator=g, device=device, dtype=torch.uint8) << 3
+    codes = (mag | sign).view(rows, K // 2, 2)
+    packed = (codes[..., 0] | (codes[..., 1] << 4)).contiguous()
+    b0 = 127 + math.floor(math.log2(1.0 / math.sqrt(fan_in))) - 2
+    sf = (b0 + torch.randint(0, 3, (rows, K // 32), generator=g, device=device)).to(torch.uint8)
+    return packed, sf
+
+
+def make_weights_mxfp4(wl: Workload, seed: int = 0, device="cpu"):
+    """MXFP4 W13 (packed [E, 2I, H/2] + scales [E, 2I, H/32]) and W2 (packed [E, H, I/2] +
+    scales [E, H, I/32]), element 2i in the low nibble of byte i."""
+    g = _gen(seed + 3, device)
+    w13p = torch.empty(wl.E, 2 * wl.I, wl.H // 2, dtype=torch.uint8, device=device)
+    w13s = torch.empty(wl.E, 2 * wl.I, wl.H // 32, dtype=torch.uint8, device=device)
+    w2p = torch.empty(wl.E, wl.H, wl.I // 2, dtype=torch.uint8, device=device)
+    w2s = torch.empty(wl.E, wl.H, wl.I // 32, dtype=torch.uint8, device=device)
+    for e in range(wl.E):
+        w13p[e], w13s[e] = _mx_block(2 * wl.I, wl.H, wl.H, g, device)
+        w2p[e], w2s[e] = _mx_block(wl.H, wl.I, wl.I, g, device)
+    return w13p, w13s, w2p, w2s
+
+
 def make_logits(wl: Workload, x: torch.Tensor, seed: int = 0) -> torch.Tensor:
     """Router logits fp32 [T, E] per the workload's routing recipe."""
     device = x.device
@@ -130,10 +163,15 @@ def make_logits(wl: Workload, x: torch.Tensor, seed: int = 0) -> torch.Tensor:
 
 
 def make_inputs(wl: Workload, seed: int = 0, device="cpu", weights: bool = True) -> dict:
+    """x, logits and the weights in the workload's format (bf16, or MXFP4 codes + scales
+    under keys w13, w13_sf, w2, w2_sf)."""
     x = make_x(wl, seed, device)
-    out = {"x": x, "logits": make_logits(wl, x, seed)}
+    out = {"x": x, "logits": make_logits(wl, x, seed), "w13_sf": None, "w2_sf": None}
     if weights:
-        out["w13"], out["w2"] = make_weights(wl, seed, device)
+        if wl.dtype == "fp8_mxfp4":
+            out["w13"], out["w13_sf"], out["w2"], out["w2_sf"] = make_weights_mxfp4(wl, seed, device)
+        else:
+            out["w13"], out["w2"] = make_weights(wl, seed, device)
     return out
 
 

@@ -104,7 +104,9 @@ def test_gemm1_fp8_parity(name):
     bound = np.abs(exact) * 2.0 ** -4 * (1 + 1e-3) + scales * 2.0 ** -10 + 1e-6 * np.abs(exact).max()
     bad = np.abs(got - exact) > bound
     assert not bad.any(), f"{bad.sum()} of {bad.size} act codes off by more than half a step"
-    assert_close(got, exact, COS_FP8, what=f"gemm1 fp8 {name}")
+    # e4m3 keeps 4 significant bits, so the requantised activation itself is only good to
+    # half a step (2^-4 of max|ref|); the 2e-2 bar applies to the layer output
+    assert_close(got, exact, COS_FP8, rel=2.0 ** -4 * 1.01, what=f"gemm1 fp8 {name}")
 
 
 @pytest.mark.parametrize("name", list(SMALL))

@@ -490,6 +490,8 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
                               const int32_t* offsets, const uint16_t* w13, uint16_t* act,
                               int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (p.I % 128 == 0 && !use_gather4() && use_pair_gemm1(p.R, p.E))
+    return launch_gemm1_bf16_2sm(p, x, row2assign, offsets, w13, act, status, stream, launches);
   const bool wide = (p.I % 128) == 0;
   const int bn = wide ? 256 : 128;
   CUtensorMap ta, tb;
@@ -522,6 +524,8 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
                               const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
                               int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (use_pair_gemm(p.R, p.E))
+    return launch_gemm2_bf16_2sm(p, act, offsets, w2, y, status, stream, launches);
   constexpr int bn = 256;
   CUtensorMap ta, tb;
   if (!make_tmap_bf16(&ta, act, p.I, p.R, BK, BM) ||

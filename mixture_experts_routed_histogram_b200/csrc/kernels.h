@@ -64,6 +64,18 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
                               const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
                               int* launches);
 
+// The same BF16 GEMMs on SM pairs (cta_group::2, 256-row tiles); use_pair_gemm decides
+// from the average rows per expert.
+bool use_pair_gemm(int64_t R, int E);
+bool use_pair_gemm1(int64_t R, int E);
+cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
+                                  const int32_t* row2assign, const int32_t* offsets,
+                                  const uint16_t* w13, uint16_t* act, int* status,
+                                  cudaStream_t stream, int* launches);
+cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
+                                  const int32_t* offsets, const uint16_t* w2, uint16_t* y,
+                                  int* status, cudaStream_t stream, int* launches);
+
 // Block-scaled grouped GEMM1 + SwiGLU + 1x128 requantisation (e4m3 x MXFP4).
 cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint32_t* sxw,
                             const int32_t* row2assign, const int32_t* offsets,

@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <algorithm>
+
 #include "kernels.h"
 #include "moe.h"
 
@@ -23,7 +25,7 @@ bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 // Workspace regions (byte offsets from the workspace base).
 struct WsLayout {
   size_t status, ids, w, counts, offsets, r2a, a2r, scratch, xq, sx, sxw, act, act_sf, act_sfw,
-      y, total;
+      y, part, total;
 };
 
 WsLayout layout(const moe_shape_t& s) {
@@ -46,6 +48,10 @@ WsLayout layout(const moe_shape_t& s) {
   L.act_sf = o; o = up(o + (fp8 ? 4 * R * (I / 128) : 0));
   L.act_sfw = o; o = up(o + (fp8 ? 4 * R * (I / 128) : 0));
   L.y = o; o = up(o + 2 * R * H);
+  // decode-sized BF16 forward: fp32 partial sums of the K-split GEMM2
+  const bool swap = !fp8 && moe::use_swap_gemm(s.T) && H % 128 == 0;
+  L.part = o;
+  o = up(o + (swap ? 4 * static_cast<size_t>(moe::kMaxSplits) * R * std::max(H, 2 * I) : 0));
   L.total = o;
   return L;
 }
@@ -304,12 +310,19 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
   const moe::GemmProblem p = problem(*shape);
   int n = 0;
   cudaError_t e;
-  if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->score,
-                             shape->renormalize, stream, &n)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if ((e = moe::launch_permute(ids, R, shape->E, counts, offsets, r2a, a2r,
-                               at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (moe::use_route_permute_small(T, shape->E, shape->k)) {
+    if ((e = moe::launch_route_permute_small(logits, T, shape->E, shape->k, shape->score,
+                                             shape->renormalize, ids, w, counts, offsets, r2a,
+                                             a2r, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  } else {
+    if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->score,
+                               shape->renormalize, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((e = moe::launch_permute(ids, R, shape->E, counts, offsets, r2a, a2r,
+                                 at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (fp8) {
     uint8_t* xq = at<uint8_t>(ws, L.xq);
     uint32_t* sxw = at<uint32_t>(ws, L.sxw);
@@ -324,6 +337,25 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     if ((e = moe::launch_gemm2_mx(p, aq, asw, offsets, static_cast<const uint8_t*>(w2), w2_sf, y,
                                   status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+  } else if (moe::use_swap_gemm(T) && shape->H % 128 == 0) {
+    // decode-sized: weights on the MMA's M side; GEMM2 splits K and the combine adds the
+    // partial sums
+    const int splits = moe::swap_splits(p);
+    float* part = at<float>(ws, L.part);  // GEMM1's partials are consumed before GEMM2's
+    if ((e = moe::launch_gemm1_swap(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+                                    part, moe::swap_splits_gemm1(p), status, stream, &n)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((e = moe::launch_gemm2_swap(p, act, offsets, static_cast<const uint16_t*>(w2), y, part,
+                                    splits, status, stream, &n)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (splits > 1) {
+      if ((e = moe::launch_combine_parts(part, splits, R, w, a2r, out, T, shape->H, shape->k,
+                                         stream, &n)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      g_last_launches = n;
+      return MOE_OK;
+    }
   } else {
     if ((e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
                                     status, stream, &n)) != cudaSuccess)

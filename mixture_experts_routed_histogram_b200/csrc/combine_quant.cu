@@ -13,6 +13,7 @@
 // Weight preparation: FlashInfer PR #6465, MXFP4 weights with K32 UE8M0 scaling; the
 // scale follows the OCP MX rule 2^(floor(log2 amax) - 2).
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -27,6 +28,8 @@ __global__ void __launch_bounds__(kCombineThreads)
   __shared__ float sw[kMaxTopK];
   __shared__ int64_t srow[kMaxTopK];
   const int64_t t = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x < k) {
     sw[threadIdx.x] = __ldg(w + t * k + threadIdx.x);
     srow[threadIdx.x] = static_cast<int64_t>(__ldg(assign2row + t * k + threadIdx.x)) * H;
@@ -58,12 +61,50 @@ __global__ void __launch_bounds__(kCombineThreads)
   }
 }
 
+// The combine when GEMM2 split K: the k rows' partial sums are added slice by slice (in
+// slice order) before the routing weights are applied (slot order), all in fp32.
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_parts_kernel(const float* __restrict__ part, int splits, int64_t R,
+                         const float* __restrict__ w, const int32_t* __restrict__ assign2row,
+                         uint16_t* __restrict__ out, int H, int k) {
+  __shared__ float sw[kMaxTopK];
+  __shared__ int64_t srow[kMaxTopK];
+  const int64_t t = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x < k) {
+    sw[threadIdx.x] = __ldg(w + t * k + threadIdx.x);
+    srow[threadIdx.x] = static_cast<int64_t>(__ldg(assign2row + t * k + threadIdx.x)) * H;
+  }
+  __syncthreads();
+  const int64_t slice = R * H;
+  for (int c = threadIdx.x * 4; c < H; c += kCombineThreads * 4) {
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int j = 0; j < k; ++j) {
+      float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int s = 0; s < splits; ++s) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(part + s * slice + srow[j] + c));
+        y[0] += v.x; y[1] += v.y; y[2] += v.z; y[3] += v.w;
+      }
+      const float wj = sw[j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(wj, y[i], acc[i]);
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    *reinterpret_cast<uint2*>(out + t * H + c) = o;
+  }
+}
+
 // One warp per (token, 128-column group); each lane owns 4 consecutive columns.
 __global__ void __launch_bounds__(256)
     quant_x_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ xq,
                    float* __restrict__ sx, uint32_t* __restrict__ sxw, int64_t groups, int H) {
   const int lane = threadIdx.x & 31;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
   if (gid >= groups) return;
   const int G = H / 128;
   const int64_t t = gid / G;
@@ -138,9 +179,17 @@ cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* ass
                            int* launches) {
   if (T == 0) return cudaSuccess;
   ++*launches;
-  combine_kernel<<<static_cast<unsigned>(T), kCombineThreads, 0, stream>>>(y, w, assign2row, out,
-                                                                           H, k);
-  return cudaGetLastError();
+  return launch_k(combine_kernel, dim3(static_cast<unsigned>(T)), dim3(kCombineThreads), 0, stream,
+                  y, w, assign2row, out, H, k);
+}
+
+cudaError_t launch_combine_parts(const float* part, int splits, int64_t R, const float* w,
+                                 const int32_t* assign2row, uint16_t* out, int64_t T, int H,
+                                 int k, cudaStream_t stream, int* launches) {
+  if (T == 0) return cudaSuccess;
+  ++*launches;
+  return launch_k(combine_parts_kernel, dim3(static_cast<unsigned>(T)), dim3(kCombineThreads), 0,
+                  stream, part, splits, R, w, assign2row, out, H, k);
 }
 
 cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* sxw, int64_t T,
@@ -148,9 +197,8 @@ cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* 
   const int64_t groups = T * (H / 128);
   if (groups == 0) return cudaSuccess;
   ++*launches;
-  quant_x_kernel<<<static_cast<unsigned>((groups + 7) / 8), 256, 0, stream>>>(x, xq, sx, sxw,
-                                                                            groups, H);
-  return cudaGetLastError();
+  return launch_k(quant_x_kernel, dim3(static_cast<unsigned>((groups + 7) / 8)), dim3(256), 0, stream,
+                  x, xq, sx, sxw, groups, H);
 }
 
 cudaError_t launch_quant_w_mxfp4(const uint16_t* w, uint8_t* packed, uint8_t* sf, int64_t rows,

@@ -36,6 +36,7 @@
 #include <string>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -136,7 +137,6 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
   const int E = args.E;
   const uint64_t lim = args.wait_limit_ns;
 
-  for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = __ldg(args.offsets + i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // cp.async mode: the B producer's expect-tx arrival + one per loader thread
@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
     tmem_alloc(s_tmem, TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {  // m-tile prefix over experts; lane l owns a contiguous expert range
     const int per = (E + 31) / 32;
@@ -410,6 +412,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
     }
   }
 
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -458,8 +461,7 @@ cudaError_t run(const CUtensorMap& a, const CUtensorMap& b, const KArgs& args,
   static cudaError_t attr = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (attr != cudaSuccess) return attr;
-  kern<<<num_sms(), threads_for(AMODE), L::ALLOC, stream>>>(a, b, args);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(num_sms()), dim3(threads_for(AMODE)), L::ALLOC, stream, a, b, args);
 }
 
 // GEMM1 A-operand path: cp.async gather (default) or TMA gather4 (MOE_GEMM1_GATHER=tma4,
@@ -490,6 +492,9 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
                               const int32_t* offsets, const uint16_t* w13, uint16_t* act,
                               int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (use_swap_gemm(p.T))
+    return launch_gemm1_swap(p, x, row2assign, offsets, w13, act, nullptr, 1, status, stream,
+                             launches);
   if (p.I % 128 == 0 && !use_gather4() && use_pair_gemm1(p.R, p.E))
     return launch_gemm1_bf16_2sm(p, x, row2assign, offsets, w13, act, status, stream, launches);
   const bool wide = (p.I % 128) == 0;
@@ -524,6 +529,8 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
                               const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
                               int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (use_swap_gemm(p.T) && p.H % 128 == 0)
+    return launch_gemm2_swap(p, act, offsets, w2, y, nullptr, 1, status, stream, launches);
   if (use_pair_gemm(p.R, p.E))
     return launch_gemm2_bf16_2sm(p, act, offsets, w2, y, status, stream, launches);
   constexpr int bn = 256;

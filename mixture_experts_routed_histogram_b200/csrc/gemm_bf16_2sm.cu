@@ -25,6 +25,7 @@
 #include <string>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -112,7 +113,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
-  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], C::FULL_COUNT);
@@ -137,6 +137,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
     tmem_alloc_2sm(s_tmem, C::TMEM_COLS);
     tmem_relinquish_2sm();
   }
+  pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {  // pair-tile prefix over experts (256 rows per pair tile)
     const int per = (E + 31) / 32;
@@ -401,6 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
     }
   }
 
+  pdl_launch_dependents();
   tc_fence_before();
   cluster_sync();  // neither CTA leaves while the pair's MMAs or signals may touch it
   if (warp == 1) {
@@ -445,8 +448,7 @@ cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const PairArgs&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
   const int grid = num_sms() & ~1;
-  kern<<<grid, Cf::THREADS, Cf::ALLOC, stream>>>(a, b, args);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(grid), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, args);
 }
 
 }  // namespace

@@ -29,6 +29,7 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -132,7 +133,6 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
   const int E = args.E;
   const uint64_t lim = args.wait_limit_ns;
 
-  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], C::FULL_COUNT);
@@ -155,6 +155,8 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     tmem_alloc(s_tmem, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {
     const int per = (E + 31) / 32;
@@ -473,6 +475,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     }
   }
 
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -485,6 +488,8 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
 __global__ void scale_words_kernel(const float* __restrict__ s, uint32_t* __restrict__ w,
                                    int64_t n) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   if (i >= n) return;
   int e;
   frexpf(__ldg(s + i), &e);  // 2^p = 0.5 * 2^(p+1)
@@ -546,8 +551,7 @@ cudaError_t run_mx(const CUtensorMap& a, const CUtensorMap& b, const MxArgs& arg
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
-  kern<<<num_sms(), Cf::THREADS, Cf::ALLOC, stream>>>(a, b, args);
-  return cudaGetLastError();
+  return launch_k(kern, dim3(num_sms()), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, args);
 }
 
 }  // namespace
@@ -556,8 +560,8 @@ cudaError_t launch_scale_words(const float* s, uint32_t* w, int64_t n, cudaStrea
                                int* launches) {
   if (n == 0) return cudaSuccess;
   ++*launches;
-  scale_words_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(s, w, n);
-  return cudaGetLastError();
+  return launch_k(scale_words_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
+                  stream, s, w, n);
 }
 
 cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint32_t* sxw,

@@ -29,6 +29,15 @@ cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t R, int E, int32_t
                                    int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                                    cudaStream_t stream, int* launches);
 
+// Routing + histogram + prefix sum + stable scatter in one single-CTA launch, for
+// decode-sized batches (use_route_permute_small).  Same outputs as launch_route followed
+// by launch_permute.
+bool use_route_permute_small(int64_t T, int E, int k);
+cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int score,
+                                       int renorm, int32_t* ids, float* w, int32_t* counts,
+                                       int32_t* offsets, int32_t* row2assign,
+                                       int32_t* assign2row, cudaStream_t stream, int* launches);
+
 // Weighted top-k combine.
 cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* assign2row,
                            uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,
@@ -75,6 +84,26 @@ cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
 cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
                                   const int32_t* offsets, const uint16_t* w2, uint16_t* y,
                                   int* status, cudaStream_t stream, int* launches);
+
+// Decode-sized GEMMs with weights on the MMA's M side and token rows on its N side.
+constexpr int kMaxSplits = 16;
+bool use_swap_gemm(int64_t T);
+int swap_splits(const GemmProblem& p);        // K slices of GEMM2
+int swap_splits_gemm1(const GemmProblem& p);  // K slices of GEMM1
+// splits == 1 fuses SwiGLU; splits > 1 writes fp32 gate|up partial sums part[splits][R][2I]
+// and a second kernel finishes act = silu(g)*u.
+cudaError_t launch_gemm1_swap(const GemmProblem& p, const uint16_t* x, const int32_t* row2assign,
+                              const int32_t* offsets, const uint16_t* w13, uint16_t* act,
+                              float* part, int splits, int* status, cudaStream_t stream,
+                              int* launches);
+// splits == 1 writes y (bf16); splits > 1 writes fp32 partial sums part[splits][R][H].
+cudaError_t launch_gemm2_swap(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
+                              const uint16_t* w2, uint16_t* y, float* part, int splits,
+                              int* status, cudaStream_t stream, int* launches);
+// Combine from K-split partial sums: out[t] = sum_j w[t,j] * sum_s part[s][assign2row[t,j]].
+cudaError_t launch_combine_parts(const float* part, int splits, int64_t R, const float* w,
+                                 const int32_t* assign2row, uint16_t* out, int64_t T, int H,
+                                 int k, cudaStream_t stream, int* launches);
 
 // Block-scaled grouped GEMM1 + SwiGLU + 1x128 requantisation (e4m3 x MXFP4).
 cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint32_t* sxw,

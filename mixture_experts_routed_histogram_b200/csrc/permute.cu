@@ -19,6 +19,8 @@
 #include <mutex>
 
 #include "kernels.h"
+#include "launch.cuh"
+#include "route_dev.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -33,6 +35,8 @@ __global__ void __launch_bounds__(kThreads)
     chunk_hist_kernel(const int32_t* __restrict__ ids, int64_t R, int E, int chunk,
                       int32_t* __restrict__ chunk_counts, int* status) {
   __shared__ int h[kMaxExperts];
+  pdl_wait();
+  pdl_launch_dependents();
   for (int e = threadIdx.x; e < E; e += kThreads) h[e] = 0;
   __syncthreads();
   const int64_t a0 = static_cast<int64_t>(blockIdx.x) * chunk;
@@ -102,6 +106,8 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ int warp_sums[kWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int me = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
 
   for (int e = tid; e < E; e += kThreads) {
     int before = 0, total = 0;
@@ -187,10 +193,142 @@ cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts
   const int chunk = chunk_size(R);
   const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
   *launches += 2;
-  chunk_hist_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, scratch, status);
-  scatter_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, nchunks, scratch, counts,
-                                                   offsets, row2assign, assign2row);
-  return cudaGetLastError();
+  cudaError_t e = launch_k(chunk_hist_kernel, dim3(nchunks), dim3(kThreads), 0, stream, ids, R, E,
+                           chunk, scratch, status);
+  if (e != cudaSuccess) return e;
+  return launch_k(scatter_kernel, dim3(nchunks), dim3(kThreads), 0, stream, ids, R, E, chunk,
+                  nchunks, static_cast<const int32_t*>(scratch), counts, offsets, row2assign,
+                  assign2row);
+}
+
+// ---------------------------------------------------------------- small batches, one launch
+//
+// For decode-sized batches (T <= 64, E <= 256) the whole front end runs in one CTA of 1024
+// threads: warps route the tokens (route_token_warp), the ids stay in shared memory, a
+// shared-memory histogram and one exclusive scan give counts/offsets, and the stable
+// scatter walks the assignments in rounds of 1024 with the same warp-match + round-stamp
+// ranking as scatter_kernel.  It replaces three launches on the latency-bound decode path.
+
+constexpr int kSmallMaxT = 64;
+constexpr int kSmallMaxE = 256;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+
+namespace {
+
+template <int VPT>
+__global__ void __launch_bounds__(kSmallThreads)
+    route_permute_small_kernel(const float* __restrict__ logits, int T, int E, int k, int score,
+                               int renorm, int32_t* __restrict__ ids, float* __restrict__ w,
+                               int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                               int32_t* __restrict__ row2assign,
+                               int32_t* __restrict__ assign2row) {
+  __shared__ int s_ids[kSmallMaxT * kMaxTopK];
+  __shared__ int scan[kSmallMaxE];
+  __shared__ int cursor[kSmallMaxE];
+  __shared__ int wcnt[kSmallWarps][kSmallMaxE];
+  __shared__ int warp_sums[kSmallWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = T * k;
+  pdl_wait();
+  pdl_launch_dependents();
+
+  for (int t = warp; t < T; t += kSmallWarps) {
+    int id;
+    float wt;
+    route_token_warp<VPT>(logits + static_cast<int64_t>(t) * E, E, k, score, renorm, lane, id,
+                          wt);
+    if (lane < k) {
+      ids[t * k + lane] = id;
+      w[t * k + lane] = wt;
+      s_ids[t * k + lane] = id;
+    }
+  }
+  for (int e = tid; e < E; e += kSmallThreads) {
+    scan[e] = 0;
+#pragma unroll 4
+    for (int ww = 0; ww < kSmallWarps; ++ww) wcnt[ww][e] = -1;
+  }
+  __syncthreads();
+  for (int a = tid; a < R; a += kSmallThreads) atomicAdd(&scan[s_ids[a]], 1);
+  __syncthreads();
+  // exclusive scan of the E counts: one per thread, warp scans, then the warp totals
+  const int cnt = tid < E ? scan[tid] : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int ww = 0; ww < warp; ++ww) before += warp_sums[ww];
+  const int excl = before + incl - cnt;
+  if (tid < E) {
+    cursor[tid] = excl;
+    offsets[tid] = excl;
+    counts[tid] = cnt;
+  }
+  if (tid == 0) offsets[E] = R;
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = 0; r * kSmallThreads < R; ++r) {
+    const int a = r * kSmallThreads + tid;
+    const int e = a < R ? s_ids[a] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt);
+    const int grp = __popc(peers);
+    const bool leader = (__ffs(peers) - 1) == lane;
+    if (e >= 0 && leader) wcnt[warp][e] = (r << 8) | grp;
+    __syncthreads();
+    if (e >= 0) {
+      int bw = 0;
+      for (int ww = 0; ww < warp; ++ww) {
+        const int v = wcnt[ww][e];
+        if ((v >> 8) == r) bw += v & 255;
+      }
+      const int row = cursor[e] + bw + rank;
+      row2assign[row] = a;
+      assign2row[a] = row;
+    }
+    __syncthreads();
+    if (e >= 0 && leader) atomicAdd(&cursor[e], grp);
+  }
+}
+
+template <int VPT>
+cudaError_t launch_small(const float* logits, int T, int E, int k, int score, int renorm,
+                         int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                         int32_t* row2assign, int32_t* assign2row, cudaStream_t stream) {
+  return launch_k(route_permute_small_kernel<VPT>, dim3(1), dim3(kSmallThreads), 0, stream, logits,
+                  T, E, k, score, renorm, ids, w, counts, offsets, row2assign, assign2row);
+}
+
+}  // namespace
+
+bool use_route_permute_small(int64_t T, int E, int k) {
+  return T > 0 && T <= kSmallMaxT && E <= kSmallMaxE && k <= kMaxTopK;
+}
+
+cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int score,
+                                       int renorm, int32_t* ids, float* w, int32_t* counts,
+                                       int32_t* offsets, int32_t* row2assign,
+                                       int32_t* assign2row, cudaStream_t stream, int* launches) {
+  ++*launches;
+  const int t = static_cast<int>(T);
+  const int need = (E + 31) / 32;
+  if (need <= 1)
+    return launch_small<1>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
+                           assign2row, stream);
+  if (need <= 2)
+    return launch_small<2>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
+                           assign2row, stream);
+  if (need <= 4)
+    return launch_small<4>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
+                           assign2row, stream);
+  return launch_small<8>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
+                         assign2row, stream);
 }
 
 // ---------------------------------------------------------------- allocation-free variant

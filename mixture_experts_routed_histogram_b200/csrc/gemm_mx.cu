@@ -570,6 +570,9 @@ cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint3
                             float* act_sf, uint32_t* act_sfw, int* status, cudaStream_t stream,
                             int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (use_mx_swap(p.R, p.E))
+    return launch_gemm1_mx_swap(p, xq, sxw, row2assign, offsets, w13p, w13sf, act, act_sf,
+                                act_sfw, status, stream, launches);
   CUtensorMap ta{}, tb;
   if (!make_tmap_fp4(&tb, w13p, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, 128))
     return cudaErrorInvalidValue;
@@ -600,6 +603,8 @@ cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint
                             const int32_t* offsets, const uint8_t* w2p, const uint8_t* w2sf,
                             uint16_t* y, int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
+  if (use_mx_swap(p.R, p.E))
+    return launch_gemm2_mx_swap(p, act, act_sfw, offsets, w2p, w2sf, y, status, stream, launches);
   CUtensorMap ta, tb;
   if (!make_tmap_u8(&ta, act, p.I, p.R, BM) ||
       !make_tmap_fp4(&tb, w2p, p.I, static_cast<uint64_t>(p.E) * p.H, 128))

@@ -117,6 +117,18 @@ cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint
                             const int32_t* offsets, const uint8_t* w2p, const uint8_t* w2sf,
                             uint16_t* y, int* status, cudaStream_t stream, int* launches);
 
+// The block-scaled GEMMs with weights on the MMA's M side, for few rows per expert
+// (use_mx_swap); same inputs and outputs as launch_gemm1_mx / launch_gemm2_mx.
+bool use_mx_swap(int64_t R, int E);
+cudaError_t launch_gemm1_mx_swap(const GemmProblem& p, const uint8_t* xq, const uint32_t* sxw,
+                                 const int32_t* row2assign, const int32_t* offsets,
+                                 const uint8_t* w13p, const uint8_t* w13sf, uint8_t* act,
+                                 float* act_sf, uint32_t* act_sfw, int* status,
+                                 cudaStream_t stream, int* launches);
+cudaError_t launch_gemm2_mx_swap(const GemmProblem& p, const uint8_t* act, const uint32_t* act_sfw,
+                                 const int32_t* offsets, const uint8_t* w2p, const uint8_t* w2sf,
+                                 uint16_t* y, int* status, cudaStream_t stream, int* launches);
+
 int num_sms();
 
 // Test hook: when non-zero, CTA 0 of each grouped-GEMM launch skips its first stage fill.

@@ -50,10 +50,12 @@ struct MxSwapArgs {
   uint64_t wait_limit_ns;
 };
 
-template <bool GEMM1, int NT, int STAGES>
+template <bool GEMM1, int NT, int STAGES, int NW2 = 1>
 struct MxSwapCfg {
   static constexpr int THREADS = 32 * 7;                 // TMA, MMA, 4 epilogue, loader
-  static constexpr int NW = GEMM1 ? 2 : 1;               // weight tiles (MMAs) per stage
+  // weight tiles (MMAs) per stage: GEMM1 the gate and up tiles; GEMM2 one or two
+  // consecutive 128-feature tiles
+  static constexpr int NW = GEMM1 ? 2 : NW2;
   static constexpr int W_BYTES = NW * BMW * BK;          // smem (codes unpacked to bytes)
   static constexpr int W_TX = NW * BMW * BK / 2;         // bytes TMA moves
   static constexpr int T_BYTES = NT * BK;                // e4m3 token rows
@@ -123,11 +125,11 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[NT]) {
   }
 }
 
-template <bool GEMM1, int NT, int STAGES>
-__global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
+template <bool GEMM1, int NT, int STAGES, int NW2>
+__global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES, NW2>::THREADS, 1)
     mx_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmT, const MxSwapArgs args) {
-  using C = MxSwapCfg<GEMM1, NT, STAGES>;
+  using C = MxSwapCfg<GEMM1, NT, STAGES, NW2>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
       int e, tt, ft;
       decode_mxs(task, s_tile, E, args.ftiles, e, tt, ft);
       const int row0 = s_off[e] + tt * NT;
-      const int wrow = e * args.w_rows + ft * BMW;
+      const int wrow = e * args.w_rows + ft * BMW * (GEMM1 ? 1 : C::NW);
       for (int kb = 0; kb < kblocks; ++kb, ++fill) {
         const int s = fill % STAGES;
         const uint32_t ph = (fill / STAGES) & 1u;
@@ -230,10 +232,14 @@ __global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], C::W_TX + (GEMM1 ? 0 : C::T_BYTES));
           tma_load_2d(w_dst, &tmW, &full[s], kb * BK, wrow);
-          if constexpr (GEMM1)
+          if constexpr (GEMM1) {
             tma_load_2d(w_dst + BMW * BK, &tmW, &full[s], kb * BK, wrow + args.n_out);  // up
-          else
+          } else {
+#pragma unroll
+            for (int w = 1; w < C::NW; ++w)
+              tma_load_2d(w_dst + w * BMW * BK, &tmW, &full[s], kb * BK, wrow + w * BMW);
             tma_load_2d(w_dst + C::W_BYTES, &tmT, &full[s], kb * BK, row0);
+          }
         }
         __syncwarp();
       }
@@ -319,7 +325,7 @@ __global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
       decode_mxs(task, s_tile, E, args.ftiles, e, tt, ft);
       const int row0 = s_off[e] + tt * NT;
       const int rows = min(NT, s_off[e + 1] - row0);
-      const int64_t wrow = static_cast<int64_t>(e) * args.w_rows + ft * BMW;
+      const int64_t wrow = static_cast<int64_t>(e) * args.w_rows + ft * BMW * (GEMM1 ? 1 : C::NW);
       const uint8_t* trow[ROWC];
       int tdst[ROWC];
       if constexpr (GEMM1) {
@@ -351,8 +357,8 @@ __global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int r = lane + 32 * j;
-            const uint8_t* src =
-                args.w_sf + (wrow + (w ? args.n_out : 0) + r) * wsf_row + kb * 4;
+            const int64_t woff = GEMM1 ? (w ? args.n_out : 0) : w * BMW;
+            const uint8_t* src = args.w_sf + (wrow + woff + r) * wsf_row + kb * 4;
             cp_async_4(sfs + 512 * w + atom_off(r), src);
           }
         // token scales: the NT rows of the tile (rows past the end reuse a valid row)
@@ -434,19 +440,23 @@ __global__ void __launch_bounds__(MxSwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
         }
         named_bar_sync_mxs(1, 128);  // red[] is rewritten by the next task
       } else {
-        uint32_t v[NT];
-        tmem_ld_n<NT>(tb, v);
+        uint32_t v[C::NW][NT];
+#pragma unroll
+        for (int w = 0; w < C::NW; ++w) tmem_ld_n<NT>(tb + w * NT, v[w]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
         uint16_t* y = static_cast<uint16_t*>(args.out);
-        const int o = ft * BMW + j;
 #pragma unroll
-        for (int c = 0; c < NT; ++c)
-          if (c < rows)
-            y[static_cast<int64_t>(row0 + c) * args.n_out + o] =
-                static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[c]), 0.0f) & 0xFFFFu);
+        for (int w = 0; w < C::NW; ++w) {
+          const int o = (ft * C::NW + w) * BMW + j;
+#pragma unroll
+          for (int c = 0; c < NT; ++c)
+            if (c < rows)
+              y[static_cast<int64_t>(row0 + c) * args.n_out + o] =
+                  static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[w][c]), 0.0f) & 0xFFFFu);
+        }
       }
       ++tc;
     }
@@ -493,27 +503,27 @@ bool tmap_mxs(CUtensorMap* m, const void* ptr, bool fp4, uint64_t inner, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GEMM1, int NT>
+template <bool GEMM1, int NT, int NW2>
 cudaError_t run_mxs(const CUtensorMap& w, const CUtensorMap& t, const MxSwapArgs& a,
                     cudaStream_t stream) {
-  using C1 = MxSwapCfg<GEMM1, NT, 1>;
+  using C1 = MxSwapCfg<GEMM1, NT, 1, NW2>;
   constexpr int STAGES0 = (190 * 1024 - C1::RED_BYTES) / (C1::STAGE + C1::SF_BYTES);
   constexpr int STAGES = STAGES0 > 8 ? 8 : STAGES0;
-  using Cf = MxSwapCfg<GEMM1, NT, STAGES>;
-  auto kern = mx_swap_gemm_kernel<GEMM1, NT, STAGES>;
+  using Cf = MxSwapCfg<GEMM1, NT, STAGES, NW2>;
+  auto kern = mx_swap_gemm_kernel<GEMM1, NT, STAGES, NW2>;
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
   return launch_k(kern, dim3(num_sms()), dim3(Cf::THREADS), Cf::ALLOC, stream, w, t, a);
 }
 
-template <bool GEMM1>
+template <bool GEMM1, int NW2>
 cudaError_t run_mxs_nt(int nt, const CUtensorMap& w, const CUtensorMap& t, const MxSwapArgs& a,
                        cudaStream_t stream) {
   switch (nt) {
-    case 16: return run_mxs<GEMM1, 16>(w, t, a, stream);
-    case 32: return run_mxs<GEMM1, 32>(w, t, a, stream);
-    default: return run_mxs<GEMM1, 64>(w, t, a, stream);
+    case 16: return run_mxs<GEMM1, 16, NW2>(w, t, a, stream);
+    case 32: return run_mxs<GEMM1, 32, NW2>(w, t, a, stream);
+    default: return run_mxs<GEMM1, 64, NW2>(w, t, a, stream);
   }
 }
 
@@ -556,7 +566,7 @@ cudaError_t launch_gemm1_mx_swap(const GemmProblem& p, const uint8_t* xq, const 
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mxs_nt<true>(mx_token_tile(p.R, p.E), tw, tt, a, stream);
+  return run_mxs_nt<true, 1>(mx_token_tile(p.R, p.E), tw, tt, a, stream);
 }
 
 cudaError_t launch_gemm2_mx_swap(const GemmProblem& p, const uint8_t* act, const uint32_t* act_sfw,
@@ -578,13 +588,17 @@ cudaError_t launch_gemm2_mx_swap(const GemmProblem& p, const uint8_t* act, const
   a.k_top = p.k;
   a.n_out = p.H;
   a.K = p.I;
-  a.ftiles = p.H / BMW;
+  // two 128-feature weight tiles per task when H allows: twice the weight bytes per stage
+  const bool pair = p.H % (2 * BMW) == 0 && nt <= 32;  // (64-row token tiles: registers)
+  a.ftiles = p.H / (pair ? 2 * BMW : BMW);
   a.w_rows = p.H;
   a.R = p.R;
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mxs_nt<false>(nt, tw, tt, a, stream);
+  if (pair) return nt == 16 ? run_mxs<false, 16, 2>(tw, tt, a, stream)
+                            : run_mxs<false, 32, 2>(tw, tt, a, stream);
+  return run_mxs_nt<false, 1>(nt, tw, tt, a, stream);
 }
 
 }  // namespace moe

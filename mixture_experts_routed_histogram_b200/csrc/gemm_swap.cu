@@ -503,8 +503,8 @@ int swap_token_tile(int64_t T) {
 bool use_swap_gemm(int64_t T) { return T <= 64; }
 
 // K slices for a decode-sized GEMM: enough (expert, feature tile, slice) tasks that the
-// last, partial wave over the SMs costs little (>= 6 waves, or >= 2 for GEMM2's fewer
-// features), counting at most min(E, R) busy experts; slices divide the K blocks and keep
+// last, partial wave over the SMs costs little (GEMM1 >= 6 waves; GEMM2 >= 2: its slices
+// are shorter and more of them measured slower), counting at most min(E, R) busy experts; slices divide the K blocks and keep
 // >= 8 blocks each.
 static int splits_for(int64_t busy_tiles, int kb, int waves) {
   int best = 1;

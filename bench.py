@@ -38,6 +38,17 @@ METRIC = "routed MoE MLP fwd TFLOP/s on 1 B200 at T=8192; µs/layer at decode T"
 # T=8192, 1 GPU: 599.60 TFLOP/s on B300 (354.38 on H200).  Context only.
 PUBLISHED = {"qwen3_30b_a3b": 599.60}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernels, from the ncu captures summarised in profiles/ (gemm_bf16_qwen3_30b_a3b_T8192,
+# gemm_swap_decode_T1, gemm_mx_swap_fp8_mxfp4_T128); an entry is removed when its kernel
+# changes after the capture.
+NCU_TRAFFIC = {
+    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 968.32e6 + 92.68e6,
+    ("qwen3_30b_a3b", 8192, "gemm2"): 503.48e6 + 238.04e6,
+    ("decode", 1, "gemm1_swiglu"): 469.82e6 + 4.16e6,
+    ("decode", 1, "gemm2"): 234.98e6 + 3.68e6,
+    ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.71e6 + 4.96e6,
+}
 
 
 def peaks():
@@ -372,7 +383,8 @@ def bench_ours(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": bytes_s[dname] / t_ker / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = NCU_TRAFFIC.get((wl.name, wl.T, dname))
+    roof["traffic_unit"] = "bytes per launch (ncu)"
     roof["kernel"] = dname
     roof["peak_source"] = (f"{pk_kind} " + ("copy" if roof["bound"] == "hbm" else
                            ("burst bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 else "burst bf16")))

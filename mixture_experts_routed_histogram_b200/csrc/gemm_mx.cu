@@ -101,8 +101,10 @@ __device__ __forceinline__ void decode_task_mx(int task, const int* s_tile, int 
   mt = local - nt * mtiles;
 }
 
+// silu(g)*u with the approximate divide: for g -> -inf the denominator overflows to +inf and
+// the quotient is 0, the limit of silu
 __device__ __forceinline__ float silu_mul_mx(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 // byte offset of row r (0..127) in a 512-byte scale atom
@@ -401,45 +403,43 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
       const bool valid = r_in < rows;
       const int64_t row = row0 + r_in;
       if constexpr (GEMM1) {
-        // pass 1: the row's amax over its 128 SwiGLU outputs
+        // one pass over the accumulator: the row's 128 SwiGLU outputs stay in registers and
+        // the accumulator goes back to the MMA warp before the requantisation and the stores
+        // (it is single-buffered, so the next tile's MMAs wait for exactly this much)
+        float a[128];
         float amax = 0.0f;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(tb + c, g);
-          tmem_ld_32x32b_x32(tb + 128 + c, u);
+#pragma unroll
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld_32x32b_x16(tb + c, g);
+          tmem_ld_32x32b_x16(tb + 128 + c, u);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            amax = fmaxf(amax, fabsf(silu_mul_mx(__uint_as_float(g[i]), __uint_as_float(u[i]))));
+          for (int i = 0; i < 16; ++i) {
+            a[c + i] = silu_mul_mx(__uint_as_float(g[i]), __uint_as_float(u[i]));
+            amax = fmaxf(amax, fabsf(a[c + i]));
+          }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
         const int se = fp8_scale_exponent(amax);
         const float inv = pow2f(-se);
-        // pass 2: e4m3 codes of act / 2^se
-        uint8_t* act = static_cast<uint8_t*>(args.out);
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(tb + c, g);
-          tmem_ld_32x32b_x32(tb + 128 + c, u);
-          tmem_ld_wait();
-          uint32_t w[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a0 = silu_mul_mx(__uint_as_float(g[4 * i + 0]), __uint_as_float(u[4 * i + 0]));
-            const float a1 = silu_mul_mx(__uint_as_float(g[4 * i + 1]), __uint_as_float(u[4 * i + 1]));
-            const float a2 = silu_mul_mx(__uint_as_float(g[4 * i + 2]), __uint_as_float(u[4 * i + 2]));
-            const float a3 = silu_mul_mx(__uint_as_float(g[4 * i + 3]), __uint_as_float(u[4 * i + 3]));
-            w[i] = static_cast<uint32_t>(cvt_e4m3x2(a0 * inv, a1 * inv)) |
-                   (static_cast<uint32_t>(cvt_e4m3x2(a2 * inv, a3 * inv)) << 16);
-          }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(act + row * args.n_out + nt * 128 + c);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          }
-        }
         if (valid) {
+          // e4m3 codes of act / 2^se: the row's 128 bytes as eight 16-byte stores
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
+                                                row * args.n_out + nt * 128);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float* p = a + 16 * v + 4 * i;
+              w[i] = static_cast<uint32_t>(cvt_e4m3x2(p[0] * inv, p[1] * inv)) |
+                     (static_cast<uint32_t>(cvt_e4m3x2(p[2] * inv, p[3] * inv)) << 16);
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
           const int64_t gi = row * (args.n_out / 128) + nt;
           if (args.out_sf) args.out_sf[gi] = pow2f(se);
           args.out_sfw[gi] = static_cast<uint32_t>(se + 127) * 0x01010101u;
@@ -463,10 +463,10 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
               dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       ++tc;
     }
     if (!ok && lane == 0) {

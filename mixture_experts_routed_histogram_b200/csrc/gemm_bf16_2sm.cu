@@ -13,8 +13,9 @@
 //   full[s]  (leader)  GEMM2: one expect-tx arrival by the leader for both CTAs' TMA bytes.
 //                      GEMM1: the same for the B halves, plus one arrival per CTA from its
 //                      relay warp once that CTA's cp.async rows of the stage have landed
-//                      (counted on the local afull[s], then forwarded at cluster scope after
-//                      a proxy fence).
+//                      (counted on the local afull[s], then forwarded to the leader after a
+//                      proxy fence, with a CTA-scope remote arrive: a cluster-scope release
+//                      there costs a fence per stage and halved the kernel's speed).
 //   empty[s] (both)    one multicast commit from the leader's MMA thread.
 //   tfull[a] (both)    one multicast commit when a tile's MMAs are done.
 //   tempty[a](leader)  one arrival per epilogue warp of either CTA (8).
@@ -276,7 +277,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
               break;
             }
             fence_async_smem();  // cp.async rows (generic proxy) -> the leader's MMA reads
-            mbar_arrive_cluster(full_leader0 + 8u * static_cast<uint32_t>(s));
+            mbar_arrive_remote(full_leader0 + 8u * static_cast<uint32_t>(s));
           }
         }
         if (!ok) {
@@ -455,9 +456,10 @@ cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const PairArgs&
 
 // Which grouped GEMMs run on SM pairs.  GEMM2 (contiguous A by TMA) does once an expert
 // averages >= 384 rows: 256-row pair tiles then waste few padded rows and halve each SM's
-// B traffic.  GEMM1 stays on single SMs: its gathered rows reach the pair leader through a
-// relay hop that measured about 2x slower than the single-SM kernel.  MOE_PAIR_GEMM=0/1
-// forces the choice for both (a tuning and test switch).
+// B traffic.  GEMM1 stays on single SMs: the pair version runs its padded work about 10 %
+// faster, but at ~500 rows per expert its 256-row tiles pad about 10 % more rows than
+// 128-row tiles, so the two measure the same.  MOE_PAIR_GEMM=0/1 forces the choice for both
+// (a tuning and test switch).
 int pair_gemm_override() {
   static const int force = [] {
     const char* e = getenv("MOE_PAIR_GEMM");

@@ -105,6 +105,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 
 // arrive (release, cluster scope) on an mbarrier given by its shared::cluster address
+// Arrive on a barrier of another CTA of the cluster with the default (CTA-scope release)
+// semantics, the form cluster pipelines use for per-stage hand-offs: unlike a cluster-scope
+// release it does not wait for this thread's view of memory to drain at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");

@@ -35,6 +35,7 @@
 #include <mutex>
 #include <string>
 
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
 #include "sm100.cuh"
@@ -81,7 +82,8 @@ struct Layout {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int OFFS_OFF = MISC_OFF + 16;
   static constexpr int TILE_OFF = OFFS_OFF + 4 * (kMaxExperts + 1);
-  static constexpr int TOTAL = TILE_OFF + 4 * (kMaxExperts + 1);
+  static constexpr int EPI_OFF = (TILE_OFF + 4 * (kMaxExperts + 1) + 1023) / 1024 * 1024;
+  static constexpr int TOTAL = EPI_OFF + kEpiBytes;  // + the epilogue's staging buffers
   static constexpr int ALLOC = TOTAL + 1024;  // slack for the 1024-byte alignment
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
@@ -102,14 +104,17 @@ __device__ __forceinline__ void decode_task(int task, const int* s_tile, int E, 
   mt = local - nt * mtiles;
 }
 
+// silu(g)*u with the approximate divide: for g -> -inf the denominator overflows to +inf and
+// the quotient is 0, the limit of silu
 __device__ __forceinline__ float silu_mul(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 template <bool GEMM1, int AMODE, int BN, int STAGES>
 __global__ void __launch_bounds__(threads_for(AMODE), 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB, const KArgs args) {
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmC, const KArgs args) {
   using L = Layout<BN, STAGES>;
   constexpr int kThreads = threads_for(AMODE);
   static_assert(GEMM1 || AMODE == kATile, "GEMM2 reads contiguous rows");
@@ -343,6 +348,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp can access
     const int r_in = q * 32 + lane;
+    EpiStager st{smem_u32(smem + L::EPI_OFF + q * kEpiWarpBytes), 0u};
     uint32_t tc = 0;
     bool ok = true;
     for (int task = blockIdx.x; task < total; task += gridDim.x) {
@@ -360,6 +366,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
       const bool valid = r_in < rows;
+      const bool whole = rows - q * 32 >= 32;  // all 32 rows of this warp are the expert's
       const int64_t row = row0 + r_in;
       if constexpr (GEMM1) {
 #pragma unroll 1
@@ -369,17 +376,17 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
           tmem_ld_32x32b_x32(tb + BN / 2 + c, u);
           tmem_ld_wait();
           const int col = nt * BN_OUT + c;
-          if (valid && col < args.n_out) {
+          if (col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                                   silu_mul(__uint_as_float(g[2 * i + 1]),
                                            __uint_as_float(u[2 * i + 1])));
-            uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.n_out + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(args.out + row * args.n_out + col, pk);
           }
         }
       } else {
@@ -389,15 +396,15 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
           tmem_ld_32x32b_x32(tb + c, v32);
           tmem_ld_wait();
           const int col = nt * BN_OUT + c;
-          if (valid && col < args.n_out) {
+          if (col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]), __uint_as_float(v32[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.n_out + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(args.out + row * args.n_out + col, pk);
           }
         }
       }
@@ -410,6 +417,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
       *s_abort = 1;
       set_status(args.status, kStatusTimeout);
     }
+    epi_drain(lane);
   }
 
   pdl_launch_dependents();
@@ -454,14 +462,14 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ou
 }
 
 template <bool GEMM1, int AMODE, int BN, int STAGES>
-cudaError_t run(const CUtensorMap& a, const CUtensorMap& b, const KArgs& args,
-                cudaStream_t stream) {
+cudaError_t run(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                const KArgs& args, cudaStream_t stream) {
   using L = Layout<BN, STAGES>;
   auto kern = grouped_gemm_bf16_kernel<GEMM1, AMODE, BN, STAGES>;
   static cudaError_t attr = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (attr != cudaSuccess) return attr;
-  return launch_k(kern, dim3(num_sms()), dim3(threads_for(AMODE)), L::ALLOC, stream, a, b, args);
+  return launch_k(kern, dim3(num_sms()), dim3(threads_for(AMODE)), L::ALLOC, stream, a, b, c, args);
 }
 
 // GEMM1 A-operand path: cp.async gather (default) or TMA gather4 (MOE_GEMM1_GATHER=tma4,
@@ -500,8 +508,10 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   const bool wide = (p.I % 128) == 0;
   const int bn = wide ? 256 : 128;
   CUtensorMap ta, tb;
+  CUtensorMap tc;
   if (!make_tmap_bf16(&ta, x, p.H, p.T, BK, 1) ||
-      !make_tmap_bf16(&tb, w13, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, BK, bn / 2))
+      !make_tmap_bf16(&tb, w13, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, BK, bn / 2) ||
+      !make_tmap_epi(encode_fn(), &tc, act, p.I, p.R))
     return cudaErrorInvalidValue;
   KArgs a{};
   a.offsets = offsets;
@@ -519,10 +529,10 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
   if (use_gather4())
-    return wide ? run<true, kAGather4, 256, 4>(ta, tb, a, stream)
-                : run<true, kAGather4, 128, 6>(ta, tb, a, stream);
-  return wide ? run<true, kACpAsync, 256, 4>(ta, tb, a, stream)
-              : run<true, kACpAsync, 128, 6>(ta, tb, a, stream);
+    return wide ? run<true, kAGather4, 256, 4>(ta, tb, tc, a, stream)
+                : run<true, kAGather4, 128, 6>(ta, tb, tc, a, stream);
+  return wide ? run<true, kACpAsync, 256, 4>(ta, tb, tc, a, stream)
+              : run<true, kACpAsync, 128, 6>(ta, tb, tc, a, stream);
 }
 
 cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
@@ -535,8 +545,10 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
     return launch_gemm2_bf16_2sm(p, act, offsets, w2, y, status, stream, launches);
   constexpr int bn = 256;
   CUtensorMap ta, tb;
+  CUtensorMap tc;
   if (!make_tmap_bf16(&ta, act, p.I, p.R, BK, BM) ||
-      !make_tmap_bf16(&tb, w2, p.I, static_cast<uint64_t>(p.E) * p.H, BK, bn))
+      !make_tmap_bf16(&tb, w2, p.I, static_cast<uint64_t>(p.E) * p.H, BK, bn) ||
+      !make_tmap_epi(encode_fn(), &tc, y, p.H, p.R))
     return cudaErrorInvalidValue;
   KArgs a{};
   a.offsets = offsets;
@@ -551,7 +563,7 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run<false, kATile, bn, 4>(ta, tb, a, stream);
+  return run<false, kATile, bn, 4>(ta, tb, tc, a, stream);
 }
 
 }  // namespace moe

@@ -25,6 +25,7 @@
 #include <mutex>
 #include <string>
 
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
 #include "sm100.cuh"
@@ -60,7 +61,8 @@ struct PairCfg {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int OFFS_OFF = MISC_OFF + 16;
   static constexpr int TILE_OFF = OFFS_OFF + 4 * (kMaxExperts + 1);
-  static constexpr int TOTAL = TILE_OFF + 4 * (kMaxExperts + 1);
+  static constexpr int EPI_OFF = (TILE_OFF + 4 * (kMaxExperts + 1) + 1023) / 1024 * 1024;
+  static constexpr int TOTAL = EPI_OFF + kEpiBytes;  // + the epilogue's staging buffers
   static constexpr int ALLOC = TOTAL + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t FULL_COUNT = GEMM1 ? 1 + 2 : 1;  // + one relay per CTA
@@ -81,14 +83,16 @@ __device__ __forceinline__ void decode_pair(int task, const int* s_tile, int E, 
   pt = local - nt * ptiles;
 }
 
+// silu(g)*u with the approximate divide (the quotient is 0 once the denominator overflows)
 __device__ __forceinline__ float silu_mul2(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 template <bool GEMM1, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGES>::THREADS, 1)
     pair_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                          const __grid_constant__ CUtensorMap tmB, const PairArgs args) {
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, const PairArgs args) {
   using C = PairCfg<GEMM1, STAGES>;
   constexpr uint32_t IDESC = idesc_bf16_f32<2 * BM, BN>();
   extern __shared__ uint8_t smem_raw[];
@@ -335,6 +339,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
     // ------------------------------------------------------------ epilogue (warps 2-5)
     const int q = warp & 3;
     const int r_in = q * 32 + lane;
+    EpiStager st{smem_u32(smem + C::EPI_OFF + q * kEpiWarpBytes), 0u};
     uint32_t tc = 0;
     bool ok = true;
     for (int task = pair; task < total; task += npairs) {
@@ -352,6 +357,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
       const bool valid = r_in < rows;
+      const bool whole = rows - q * 32 >= 32;  // all 32 rows of this warp are the expert's
       const int64_t row = row0 + r_in;
       if constexpr (GEMM1) {
 #pragma unroll 1
@@ -361,17 +367,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
           tmem_ld_32x32b_x32(tb + BN / 2 + c, u);
           tmem_ld_wait();
           const int col = nt * (BN / 2) + c;
-          if (valid && col < args.n_out) {
+          if (col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(silu_mul2(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                                   silu_mul2(__uint_as_float(g[2 * i + 1]),
                                             __uint_as_float(u[2 * i + 1])));
-            uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.n_out + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(args.out + row * args.n_out + col, pk);
           }
         }
       } else {
@@ -381,15 +387,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
           tmem_ld_32x32b_x32(tb + c, v32);
           tmem_ld_wait();
           const int col = nt * BN + c;
-          if (valid && col < args.n_out) {
+          if (col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]), __uint_as_float(v32[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(args.out + row * args.n_out + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(args.out + row * args.n_out + col, pk);
           }
         }
       }
@@ -402,6 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
       *s_abort = 1;
       set_status(args.status, kStatusTimeout);
     }
+    epi_drain(lane);
   }
 
   pdl_launch_dependents();
@@ -441,15 +448,15 @@ bool tmap_bf16_2sm(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
 }
 
 template <bool GEMM1, int STAGES>
-cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const PairArgs& args,
-                     cudaStream_t stream) {
+cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                     const PairArgs& args, cudaStream_t stream) {
   using Cf = PairCfg<GEMM1, STAGES>;
   auto kern = pair_gemm_bf16_kernel<GEMM1, STAGES>;
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
   const int grid = num_sms() & ~1;
-  return launch_k(kern, dim3(grid), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, args);
+  return launch_k(kern, dim3(grid), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, c, args);
 }
 
 }  // namespace
@@ -484,8 +491,9 @@ cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
                                   cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
   if (p.I % 128 != 0) return cudaErrorInvalidValue;
-  CUtensorMap ta{}, tb;
-  if (!tmap_bf16_2sm(&tb, w13, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, BN / 2))
+  CUtensorMap ta{}, tb, tc;
+  if (!tmap_bf16_2sm(&tb, w13, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, BN / 2) ||
+      !make_tmap_epi(encode_fn_2sm(), &tc, act, p.I, p.R))
     return cudaErrorInvalidValue;
   PairArgs a{};
   a.offsets = offsets;
@@ -502,16 +510,17 @@ cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_pair<true, 6>(ta, tb, a, stream);
+  return run_pair<true, 6>(ta, tb, tc, a, stream);
 }
 
 cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
                                   const int32_t* offsets, const uint16_t* w2, uint16_t* y,
                                   int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!tmap_bf16_2sm(&ta, act, p.I, p.R, BM) ||
-      !tmap_bf16_2sm(&tb, w2, p.I, static_cast<uint64_t>(p.E) * p.H, BN / 2))
+      !tmap_bf16_2sm(&tb, w2, p.I, static_cast<uint64_t>(p.E) * p.H, BN / 2) ||
+      !make_tmap_epi(encode_fn_2sm(), &tc, y, p.H, p.R))
     return cudaErrorInvalidValue;
   PairArgs a{};
   a.offsets = offsets;
@@ -526,7 +535,7 @@ cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_pair<false, 6>(ta, tb, a, stream);
+  return run_pair<false, 6>(ta, tb, tc, a, stream);
 }
 
 }  // namespace moe

@@ -115,11 +115,10 @@ MOE_API moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, i
  * start-up and which has no scratch buffer to pass down.  (This entry point has no
  * counterpart on the pages; it is a packaging variant of the permutation above.)
  * Same inputs, outputs and results as moe_permute, bit for bit.  The per-chunk
- * histograms live in a 256 KB file-scope device array instead of the workspace; it
- * needs ceil(T*k / chunk) * E <= 65536, where chunk = 2048 while T*k <= 524288 (so
- * E = 512 works up to T*k = 262144 and E = 128 up to 524288; beyond 524288 the chunk
- * grows so that there are 256 chunks, which needs E <= 256).  Larger problems return
- * MOE_ERR_UNSUPPORTED_SHAPE without launching anything.  The first call on each device
+ * histograms and their scans live in a 512 KB file-scope device array instead of the
+ * workspace; it needs (2 * nch + 1) * E <= 131072 ints, where nch = ceil(T / 64) up to
+ * T = 8192 and 128 beyond (the chunks grow), so every T works for E <= 510.  Larger
+ * problems return MOE_ERR_UNSUPPORTED_SHAPE without launching anything.  The first call on each device
  * looks up the array's device address (cudaGetSymbolAddress, with that device current);
  * make that first call before any stream capture.  Every call shares the array: calls
  * whose kernels overlap on the GPU (other streams, other host threads) race on it;

@@ -40,7 +40,7 @@ WsLayout layout(const moe_shape_t& s) {
   L.offsets = o; o = up(o + 4 * (E + 1));
   L.r2a = o; o = up(o + 4 * R);
   L.a2r = o; o = up(o + 4 * R);
-  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(R), s.E));
+  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(T), s.E));
   L.xq = o; o = up(o + (fp8 ? T * H : 0));
   L.sx = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
   L.sxw = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
@@ -147,11 +147,12 @@ moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* ids, int32_t* 
   const int64_t R = shape->T * shape->k;
   if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
   const WsLayout L = layout(*shape);
-  if (ws_bytes < L.scratch + moe::permute_scratch_bytes(R, shape->E))
+  if (ws_bytes < L.scratch + moe::permute_scratch_bytes(shape->T, shape->E))
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   int n = 0;
-  cudaError_t e = moe::launch_permute(ids, R, shape->E, counts, offsets, row2assign, assign2row,
-                                      at<int32_t>(ws, L.scratch), status_word(ws), stream, &n);
+  cudaError_t e = moe::launch_permute(ids, shape->T, shape->k, shape->E, counts, offsets,
+                                      row2assign, assign2row, at<int32_t>(ws, L.scratch),
+                                      status_word(ws), stream, &n);
   g_last_launches = n;
   return cuda_status(e);
 }
@@ -164,10 +165,10 @@ moe_status_t moe_permute_noalloc(const moe_shape_t* shape, const int32_t* ids, i
   MOE_TRY(need_ptrs({counts, offsets}));
   const int64_t R = shape->T * shape->k;
   if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
-  if (!moe::permute_noalloc_fits(R, shape->E)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!moe::permute_noalloc_fits(shape->T, shape->E)) return MOE_ERR_UNSUPPORTED_SHAPE;
   int n = 0;
-  cudaError_t e = moe::launch_permute_noalloc(ids, R, shape->E, counts, offsets, row2assign,
-                                              assign2row, stream, &n);
+  cudaError_t e = moe::launch_permute_noalloc(ids, shape->T, shape->k, shape->E, counts, offsets,
+                                              row2assign, assign2row, stream, &n);
   g_last_launches = n;
   return cuda_status(e);
 }
@@ -319,7 +320,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->score,
                                shape->renormalize, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if ((e = moe::launch_permute(ids, R, shape->E, counts, offsets, r2a, a2r,
+    if ((e = moe::launch_permute(ids, T, shape->k, shape->E, counts, offsets, r2a, a2r,
                                  at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }

@@ -16,16 +16,18 @@ constexpr int kMaxTopK = 32;
 cudaError_t launch_route(const float* logits, int32_t* ids, float* w, int64_t T, int E, int k,
                          int score, int renorm, cudaStream_t stream, int* launches);
 
-// Histogram / prefix sum / stable scatter.  `scratch` holds the per-chunk histograms.
-size_t permute_scratch_bytes(int64_t R, int E);
-cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts,
+// Histogram / prefix sum / stable scatter of the T*k assignments (chunks of 64 tokens,
+// fewer and larger chunks beyond 128 of them).  `scratch` holds the per-chunk histograms
+// and their scans.
+size_t permute_scratch_bytes(int64_t T, int E);
+cudaError_t launch_permute(const int32_t* ids, int64_t T, int k, int E, int32_t* counts,
                            int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                            int32_t* scratch, int* status, cudaStream_t stream, int* launches);
 
-// The same permutation with its per-chunk histograms in a static device array (no
-// workspace); fits() tells whether ceil(R / chunk) * E stays within that array.
-bool permute_noalloc_fits(int64_t R, int E);
-cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t R, int E, int32_t* counts,
+// The same permutation with its scratch in a static device array (no workspace); fits()
+// tells whether the problem's scratch stays within that array.
+bool permute_noalloc_fits(int64_t T, int E);
+cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t T, int k, int E, int32_t* counts,
                                    int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                                    cudaStream_t stream, int* launches);
 

@@ -6,16 +6,19 @@
 // listed change: a flat m-task queue replaces a per-tile rescan of the experts; the
 // offsets produced here are what the GEMM kernels turn into that queue.
 //
-// Two launches, both deterministic (no atomics decide an order):
-//   1. chunk_hist_kernel: one CTA per chunk of consecutive assignments counts the
-//      assignments of each expert in its chunk (shared-memory histogram).
-//   2. scatter_kernel:    one CTA per chunk reads every chunk's histogram (a few hundred
-//      KB at most, L2-resident), forms offsets[e] = exclusive scan over experts of the
-//      totals, and the chunk's starting row for each expert = offsets[e] + the counts of
-//      the earlier chunks.  It then walks its chunk in order, 256 assignments per round,
-//      ranking equal experts inside a warp with __match_any_sync and across the 8 warps
-//      with round-stamped per-warp counts, so the row of assignment a is offsets[e] +
-//      #{a' < a : ids[a'] == e}: the stable order.
+// Three launches, all deterministic (no atomics decide an order).  Chunks are 64 tokens'
+// assignments (larger once there would be more than 128 chunks), so each launch has one CTA
+// per chunk or per expert and every SM has work at T = 8192:
+//   1. chunk_hist_kernel: one CTA per chunk counts the assignments of each expert in its
+//      chunk (shared-memory histogram) into cc[e][chunk].
+//   2. chunk_scan_kernel: one CTA per expert scans its row of cc over the chunks:
+//      base[e][chunk] = the expert's assignments in earlier chunks, tot[e] = all of them.
+//   3. scatter_kernel:    one CTA per chunk forms offsets[e] = exclusive scan over experts of
+//      tot, so the chunk's first row for expert e is offsets[e] + base[e][chunk].  It then
+//      walks its chunk in order, 256 assignments per round, ranking equal experts inside a
+//      warp with __match_any_sync and across the 8 warps with round-stamped per-warp
+//      counts, so the row of assignment a is offsets[e] + #{a' < a : ids[a'] == e}: the
+//      stable order.
 #include <mutex>
 
 #include "kernels.h"
@@ -28,12 +31,31 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kDefaultChunk = 2048;
-constexpr int kMaxChunks = 256;
+constexpr int kMaxChunks = 128;          // chunks per call (one scan CTA thread each)
+constexpr int kMinChunkTokens = 64;
 
+// Tokens per chunk: 64, doubled until there are at most kMaxChunks chunks.
+int chunk_tokens(int64_t T) {
+  int64_t t = kMinChunkTokens;
+  while ((T + t - 1) / t > kMaxChunks) t *= 2;
+  return static_cast<int>(t);
+}
+
+int num_chunks(int64_t T) {
+  const int64_t t = chunk_tokens(T);
+  return T > 0 ? static_cast<int>((T + t - 1) / t) : 1;
+}
+
+// Scratch: per-chunk counts cc[E][nch], their exclusive scan over chunks base[E][nch], and
+// the expert totals tot[E] (ints).
+size_t scratch_ints(int64_t T, int E) {
+  return static_cast<size_t>(2) * E * num_chunks(T) + E;
+}
+
+// Histogram of one chunk of consecutive assignments: cc[e][chunk].
 __global__ void __launch_bounds__(kThreads)
-    chunk_hist_kernel(const int32_t* __restrict__ ids, int64_t R, int E, int chunk,
-                      int32_t* __restrict__ chunk_counts, int* status) {
+    chunk_hist_kernel(const int32_t* __restrict__ ids, int64_t R, int E, int chunk, int nch,
+                      int32_t* __restrict__ cc, int* status) {
   __shared__ int h[kMaxExperts];
   pdl_wait();
   pdl_launch_dependents();
@@ -45,12 +67,12 @@ __global__ void __launch_bounds__(kThreads)
     const int e = __ldg(ids + a);
     if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
       atomicAdd(&h[e], 1);
-    else
+    else if (status)
       set_status(status, kStatusBadIndex);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kThreads)
-    chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = h[e];
+    cc[static_cast<int64_t>(e) * nch + blockIdx.x] = h[e];
 }
 
 // In-place exclusive scan of s[0..n) (n <= 4 * kThreads) by the whole block; returns
@@ -95,32 +117,48 @@ __device__ int block_exclusive_scan(int* s, int n, int* warp_sums) {
   return total;
 }
 
+// One CTA per expert: base[e][c] = sum of cc[e][c'] over the chunks c' < c, tot[e] = all.
 __global__ void __launch_bounds__(kThreads)
-    scatter_kernel(const int32_t* __restrict__ ids, int64_t R, int E, int chunk, int nchunks,
-                   const int32_t* __restrict__ chunk_counts, int32_t* __restrict__ counts,
-                   int32_t* __restrict__ offsets, int32_t* __restrict__ row2assign,
-                   int32_t* __restrict__ assign2row) {
+    chunk_scan_kernel(const int32_t* __restrict__ cc, int nch, int32_t* __restrict__ base,
+                      int32_t* __restrict__ tot) {
+  __shared__ int s[kThreads];
+  __shared__ int warp_sums[kWarps];
+  const int e = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  s[tid] = tid < nch ? __ldg(cc + static_cast<int64_t>(e) * nch + tid) : 0;
+  __syncthreads();
+  const int total = block_exclusive_scan(s, nch, warp_sums);
+  if (tid < nch) base[static_cast<int64_t>(e) * nch + tid] = s[tid];
+  if (tid == 0) tot[e] = total;
+}
+
+// One CTA per chunk: offsets[e] = exclusive scan over experts of tot[e]; the chunk's first
+// row for expert e is offsets[e] + base[e][chunk].  The chunk is then walked in order, 256
+// assignments per round, ranking equal experts inside a warp with __match_any_sync and
+// across the 8 warps with round-stamped per-warp counts, so the row of assignment a is
+// offsets[e] + #{a' < a : ids[a'] == e}: the stable order.
+__global__ void __launch_bounds__(kThreads)
+    scatter_kernel(const int32_t* __restrict__ ids, int64_t R, int E, int chunk, int nch,
+                   const int32_t* __restrict__ base, const int32_t* __restrict__ tot,
+                   int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ row2assign, int32_t* __restrict__ assign2row) {
   __shared__ int cursor[kMaxExperts];
   __shared__ int scan[kMaxExperts];
   __shared__ int wcnt[kWarps][kMaxExperts];
   __shared__ int warp_sums[kWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int me = blockIdx.x;
+  for (int e = tid; e < E; e += kThreads) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) wcnt[w][e] = -1;
+  }
   pdl_wait();
   pdl_launch_dependents();
 
   for (int e = tid; e < E; e += kThreads) {
-    int before = 0, total = 0;
-#pragma unroll 8
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = __ldg(chunk_counts + static_cast<int64_t>(c) * E + e);
-      total += v;
-      before += (c < me) ? v : 0;
-    }
-    cursor[e] = before;
-    scan[e] = total;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) wcnt[w][e] = -1;
+    cursor[e] = __ldg(base + static_cast<int64_t>(e) * nch + me);
+    scan[e] = __ldg(tot + e);
   }
   __syncthreads();
   const int grand = block_exclusive_scan(scan, E, warp_sums);
@@ -165,40 +203,49 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-int chunk_size(int64_t R) {
-  int64_t c = kDefaultChunk;
-  if ((R + c - 1) / c > kMaxChunks) {
-    c = (R + kMaxChunks - 1) / kMaxChunks;
-    c = (c + kThreads - 1) / kThreads * kThreads;
-  }
-  return static_cast<int>(c);
+// Scan + scatter after the chunk histograms are in `scratch`.
+cudaError_t launch_scan_scatter(const int32_t* ids, int64_t T, int k, int E, int32_t* counts,
+                                int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                int32_t* scratch, cudaStream_t stream, int* launches) {
+  const int tpc = chunk_tokens(T);
+  const int nch = num_chunks(T);
+  const int64_t R = T * k;
+  int32_t* cc = scratch;
+  int32_t* base = cc + static_cast<int64_t>(E) * nch;
+  int32_t* tot = base + static_cast<int64_t>(E) * nch;
+  *launches += 2;
+  cudaError_t e = launch_k(chunk_scan_kernel, dim3(E), dim3(kThreads), 0, stream,
+                           static_cast<const int32_t*>(cc), nch, base, tot);
+  if (e != cudaSuccess) return e;
+  return launch_k(scatter_kernel, dim3(nch), dim3(kThreads), 0, stream, ids, R, E, tpc * k, nch,
+                  static_cast<const int32_t*>(base), static_cast<const int32_t*>(tot), counts,
+                  offsets, row2assign, assign2row);
+}
+
+cudaError_t permute_empty(int E, int32_t* counts, int32_t* offsets, cudaStream_t stream,
+                          int* launches) {
+  ++*launches;
+  cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
+  if (e != cudaSuccess) return e;
+  return cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
 }
 
 }  // namespace
 
-size_t permute_scratch_bytes(int64_t R, int E) {
-  const int64_t c = chunk_size(R);
-  const int64_t n = R > 0 ? (R + c - 1) / c : 1;
-  return static_cast<size_t>(n) * E * sizeof(int32_t);
-}
+size_t permute_scratch_bytes(int64_t T, int E) { return scratch_ints(T, E) * sizeof(int32_t); }
 
-cudaError_t launch_permute(const int32_t* ids, int64_t R, int E, int32_t* counts,
+cudaError_t launch_permute(const int32_t* ids, int64_t T, int k, int E, int32_t* counts,
                            int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                            int32_t* scratch, int* status, cudaStream_t stream, int* launches) {
-  if (R == 0) {
-    ++*launches;
-    cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
-    return cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
-  }
-  const int chunk = chunk_size(R);
-  const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
-  *launches += 2;
-  cudaError_t e = launch_k(chunk_hist_kernel, dim3(nchunks), dim3(kThreads), 0, stream, ids, R, E,
-                           chunk, scratch, status);
+  if (T == 0) return permute_empty(E, counts, offsets, stream, launches);
+  const int tpc = chunk_tokens(T);
+  const int nch = num_chunks(T);
+  ++*launches;
+  cudaError_t e = launch_k(chunk_hist_kernel, dim3(nch), dim3(kThreads), 0, stream, ids, T * k, E,
+                           tpc * k, nch, scratch, status);
   if (e != cudaSuccess) return e;
-  return launch_k(scatter_kernel, dim3(nchunks), dim3(kThreads), 0, stream, ids, R, E, chunk,
-                  nchunks, static_cast<const int32_t*>(scratch), counts, offsets, row2assign,
-                  assign2row);
+  return launch_scan_scatter(ids, T, k, E, counts, offsets, row2assign, assign2row, scratch,
+                             stream, launches);
 }
 
 // ---------------------------------------------------------------- small batches, one launch
@@ -333,14 +380,14 @@ cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, in
 
 // ---------------------------------------------------------------- allocation-free variant
 //
-// For callers that cannot hand the library a workspace: the per-chunk histograms live in
-// this file-scope device array instead (256 KB, held on every device that loads the
-// library until the process exits).  Every call shares it, so two calls whose kernels
-// overlap on the GPU (different streams, or different host threads) race on it; calls
-// serialised on one stream are safe.  The histogram kernel overwrites every entry a call
-// reads, so nothing has to be cleared between calls.
+// For callers that cannot hand the library a workspace: the per-chunk histograms and their
+// scans live in this file-scope device array instead (512 KB, held on every device that
+// loads the library until the process exits).  Every call shares it, so two calls whose
+// kernels overlap on the GPU (different streams, or different host threads) race on it;
+// calls serialised on one stream are safe.  The kernels overwrite every entry a call reads,
+// so nothing has to be cleared between calls.
 
-constexpr int kNoAllocScratchInts = 1 << 16;
+constexpr int kNoAllocScratchInts = 1 << 17;
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 
 namespace {
@@ -368,31 +415,19 @@ static cudaError_t noalloc_scratch(int32_t** out) {
   return cudaSuccess;
 }
 
-bool permute_noalloc_fits(int64_t R, int E) {
-  if (R == 0) return true;
-  const int64_t c = chunk_size(R);
-  const int64_t n = (R + c - 1) / c;
-  return n * E <= kNoAllocScratchInts;
+bool permute_noalloc_fits(int64_t T, int E) {
+  return T == 0 || scratch_ints(T, E) <= static_cast<size_t>(kNoAllocScratchInts);
 }
 
-cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t R, int E, int32_t* counts,
+cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t T, int k, int E, int32_t* counts,
                                    int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
                                    cudaStream_t stream, int* launches) {
-  if (R == 0) {
-    ++*launches;
-    cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream);
-    return cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream);
-  }
+  if (T == 0) return permute_empty(E, counts, offsets, stream, launches);
   int32_t* scratch = nullptr;
   cudaError_t e = noalloc_scratch(&scratch);
   if (e != cudaSuccess) return e;
-  const int chunk = chunk_size(R);
-  const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
-  *launches += 2;
-  chunk_hist_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, scratch, nullptr);
-  scatter_kernel<<<nchunks, kThreads, 0, stream>>>(ids, R, E, chunk, nchunks, scratch, counts,
-                                                   offsets, row2assign, assign2row);
-  return cudaGetLastError();
+  return launch_permute(ids, T, k, E, counts, offsets, row2assign, assign2row, scratch, nullptr,
+                        stream, launches);
 }
 
 }  // namespace moe

@@ -203,6 +203,19 @@ def test_forward_skewed_one_expert():
     _check_forward(wl, inp, _skewed_logits(wl, inp["x"]), np.arange(wl.T))
 
 
+@pytest.mark.parametrize("wl", [I.Workload("ties", 300, 256, 128, 64, 4),
+                                I.Workload("wide", 100, 256, 128, 1000, 32, routing="uniform")],
+                         ids=["ties_e64_k4", "e1000_k32"])
+def test_forward_front_end_ties_and_wide_routing(wl):
+    """The large-batch front end of moe_forward (routing fused with the chunk histograms,
+    scan, scatter): coarse logits with many exact ties, and 1000 experts with top-32."""
+    inp = I.make_inputs(wl, 0, dev())
+    lg = inp["logits"]
+    if wl.name == "ties":
+        lg = torch.round(lg * 2) / 2
+    _check_forward(wl, inp, lg, np.arange(wl.T))
+
+
 def test_forward_deterministic():
     wl = SMALL["many_tiles"]
     inp = I.make_inputs(wl, 0, dev())

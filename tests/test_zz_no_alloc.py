@@ -47,7 +47,7 @@ def test_noalloc_permute_matches_workspace_permute_twice(T, k, E):
 
 
 def test_noalloc_permute_rejects_sizes_beyond_its_scratch():
-    shape = C.MoeShape.of(60000, 256, 128, 1024, 10)   # 235 chunks x 1024 experts > 65536
+    shape = C.MoeShape.of(60000, 256, 128, 1024, 10)   # (2 * 128 + 1) * 1024 ints > 131072
     E, R = 1024, 600000
     with pytest.raises(C.MoeError) as ex:
         C.moe_permute_noalloc(shape, torch.zeros(R, dtype=torch.int32, device="cuda"),

@@ -461,12 +461,12 @@ cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
 
 }  // namespace
 
-// Which grouped GEMMs run on SM pairs.  GEMM2 (contiguous A by TMA) does once an expert
-// averages >= 384 rows: 256-row pair tiles then waste few padded rows and halve each SM's
-// B traffic.  GEMM1 stays on single SMs: the pair version runs its padded work about 10 %
-// faster, but at ~500 rows per expert its 256-row tiles pad about 10 % more rows than
-// 128-row tiles, so the two measure the same.  MOE_PAIR_GEMM=0/1 forces the choice for both
-// (a tuning and test switch).
+// Which grouped GEMMs run on SM pairs.  The pair kernels run their padded work about 10 %
+// faster than the single-SM ones (half the B bytes per SM), but their 256-row tiles pad
+// more rows: at ~500 rows per expert 20 % against 11 %, a wash in time and more energy
+// under the power cap.  So GEMM2 (contiguous A by TMA) pairs only once an expert averages
+// >= 768 rows, and GEMM1 (whose gathered A reaches the leader through a relay warp) stays
+// on single SMs.  MOE_PAIR_GEMM=0/1 forces the choice for both (a tuning and test switch).
 int pair_gemm_override() {
   static const int force = [] {
     const char* e = getenv("MOE_PAIR_GEMM");
@@ -477,7 +477,7 @@ int pair_gemm_override() {
 
 bool use_pair_gemm(int64_t R, int E) {
   if (pair_gemm_override() >= 0) return pair_gemm_override() != 0;
-  return R >= static_cast<int64_t>(E) * 384;
+  return R >= static_cast<int64_t>(E) * 768;
 }
 
 bool use_pair_gemm1(int64_t R, int E) {

@@ -28,6 +28,7 @@
 
 #include <mutex>
 
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "launch.cuh"
 #include "sm100.cuh"
@@ -76,12 +77,16 @@ struct MxCfg {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int OFFS_OFF = MISC_OFF + 16;
   static constexpr int TILE_OFF = OFFS_OFF + 4 * (kMaxExperts + 1);
-  static constexpr int TOTAL = TILE_OFF + 4 * (kMaxExperts + 1);
+  // GEMM2 stages its bf16 output through per-warp buffers for TMA stores
+  static constexpr int EPI_OFF = (TILE_OFF + 4 * (kMaxExperts + 1) + 1023) / 1024 * 1024;
+  static constexpr int TOTAL = EPI_OFF + (GEMM1 ? 0 : kEpiBytes);
   static constexpr int ALLOC = TOTAL + 1024;
   static constexpr int SF_COLS = 4 + BN / 32;        // TMEM columns per stage: SFA + SFB
   static constexpr int SF_TMEM = NACC * BN;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t FULL_COUNT = 1 + (GEMM1 ? 32 * kLoaderWarps : 32);
+  // expect-tx arrival + per loader thread: GEMM1 a cp.async arrival and a store arrival,
+  // GEMM2 (one scale warp) a cp.async arrival
+  static constexpr uint32_t FULL_COUNT = 1 + (GEMM1 ? 2 * 32 * kLoaderWarps : 32);
   static_assert(STAGE % 1024 == 0, "stage alignment");
   static_assert(SF_TMEM + STAGES * SF_COLS <= static_cast<int>(TMEM_COLS), "TMEM budget");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
@@ -113,7 +118,8 @@ __device__ __forceinline__ int sf_atom_off(int r) { return 16 * (r & 31) + 4 * (
 template <bool GEMM1, int STAGES>
 __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     mx_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const MxArgs args) {
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmC, const MxArgs args) {
   using C = MxCfg<GEMM1, STAGES>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -296,12 +302,19 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     uint32_t fill = 0;
     bool ok = true;
     if constexpr (GEMM1) {
-      // A rows (e4m3) + the stage's scale atoms: 128 threads, thread t owns scale row t
+      // A rows (e4m3) + the stage's scale atoms: 128 threads, thread t owns scale row t.
+      // The rows go by 16-byte cp.async (tracked by the no-increment arrival); the scale
+      // words of the thread's three rows (token row of A, gate and up rows of B) are read
+      // with plain loads one group of 4 stages ahead, written into the stage's atoms with
+      // st.shared and published by a second, regular arrival after a proxy fence.
       const int lw = warp - 6;
       const int sub = lane >> 3;
       const int chunk = lane & 7;
       const int t = lw * 32 + lane;
-      const int G = args.K / 128;
+      const int G = args.K / 128;          // scale words per row (one per K=128 stage)
+      // rows start on 16 bytes (4 words per load) when G % 4 == 0 and both bases are aligned
+      const bool vec = (G & 3) == 0 && ((reinterpret_cast<uintptr_t>(args.a_sfw) |
+                                         reinterpret_cast<uintptr_t>(args.b_sf)) & 15u) == 0;
       for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
         int e, mt, nt;
         decode_task_mx(task, s_tile, E, args.n_tiles, e, mt, nt);
@@ -315,12 +328,29 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
           src[i] = args.a_rows + static_cast<int64_t>(tok) * args.K + chunk * 16;
         }
         const int tok_t = __ldg(args.row2assign + row0 + (t < rows ? t : 0)) / args.k_top;
-        const uint32_t* sfa_src = args.a_sfw + static_cast<int64_t>(tok_t) * G;
         const int64_t brow = static_cast<int64_t>(e) * args.b_rows + nt * C::BN_OUT;
-        const uint8_t* sfg_src = args.b_sf + (brow + t) * sf_row_bytes;
-        const uint8_t* sfu_src = args.b_sf + (brow + args.n_out + t) * sf_row_bytes;
+        const uint32_t* wrow[3] = {
+            args.a_sfw + static_cast<int64_t>(tok_t) * G,
+            reinterpret_cast<const uint32_t*>(args.b_sf + (brow + t) * sf_row_bytes),
+            reinterpret_cast<const uint32_t*>(args.b_sf + (brow + args.n_out + t) * sf_row_bytes)};
+        uint32_t cw[3][4], nw[3][4];
+        auto load_group = [&](int g0, uint32_t (&w)[3][4]) {
+#pragma unroll
+          for (int r = 0; r < 3; ++r) {
+            if (vec) {
+              const uint4 v = __ldg(reinterpret_cast<const uint4*>(wrow[r] + g0));
+              w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) w[r][j] = g0 + j < G ? __ldg(wrow[r] + g0 + j) : 0u;
+            }
+          }
+        };
+        load_group(0, cw);
         const int sfo = sf_atom_off(t);
         for (int kb = 0; kb < kblocks; ++kb, ++fill) {
+          const int gi = kb & 3;
+          if (gi == 0 && kb + 4 < kblocks) load_group(kb + 4, nw);
           const int s = fill % STAGES;
           const uint32_t ph = (fill / STAGES) & 1u;
           if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, s_abort, lim))) {
@@ -334,10 +364,20 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
             cp_async_16(a_base + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * BK);
           }
           const uint32_t sf_base = smem_u32(smem + C::SF_OFF + s * C::SF_BYTES);
-          cp_async_4(sf_base + sfo, sfa_src + kb);
-          cp_async_4(sf_base + 512 + sfo, sfg_src + kb * 4);
-          cp_async_4(sf_base + 1024 + sfo, sfu_src + kb * 4);
+#pragma unroll
+          for (int r = 0; r < 3; ++r) {
+            const uint32_t v = gi == 0 ? cw[r][0] : gi == 1 ? cw[r][1] : gi == 2 ? cw[r][2] : cw[r][3];
+            st_shared_b32(sf_base + 512 * r + sfo, v);
+          }
+          fence_async_smem();  // the atom words (generic proxy) -> tcgen05.cp (async proxy)
           cp_async_mbar_arrive_noinc(&full[s]);
+          mbar_arrive(&full[s]);
+          if (gi == 3) {
+#pragma unroll
+            for (int r = 0; r < 3; ++r)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) cw[r][j] = nw[r][j];
+          }
         }
       }
     } else {
@@ -384,6 +424,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     // ------------------------------------------------------------ epilogue (warps 2-5)
     const int q = warp & 3;
     const int r_in = q * 32 + lane;
+    EpiStager st{smem_u32(smem + C::EPI_OFF + q * kEpiWarpBytes), 0u};
     uint32_t tc = 0;
     bool ok = true;
     for (int task = blockIdx.x; task < total; task += gridDim.x) {
@@ -401,6 +442,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
       const bool valid = r_in < rows;
+      const bool whole = rows - q * 32 >= 32;  // all 32 rows of this warp are the expert's
       const int64_t row = row0 + r_in;
       if constexpr (GEMM1) {
         // one pass over the accumulator: the row's 128 SwiGLU outputs stay in registers and
@@ -452,15 +494,15 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
           tmem_ld_32x32b_x32(tb + c, v32);
           tmem_ld_wait();
           const int col = nt * C::BN_OUT + c;
-          if (valid && col < args.n_out) {
+          if (col < args.n_out) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]), __uint_as_float(v32[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(y + row * args.n_out + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(y + row * args.n_out + col, pk);
           }
         }
         tc_fence_before();
@@ -473,6 +515,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
       *s_abort = 1;
       set_status(args.status, kStatusTimeout);
     }
+    if constexpr (!GEMM1) epi_drain(lane);
   }
 
   pdl_launch_dependents();
@@ -544,14 +587,14 @@ bool make_tmap_fp4(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
 }
 
 template <bool GEMM1, int STAGES>
-cudaError_t run_mx(const CUtensorMap& a, const CUtensorMap& b, const MxArgs& args,
-                   cudaStream_t stream) {
+cudaError_t run_mx(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                   const MxArgs& args, cudaStream_t stream) {
   using Cf = MxCfg<GEMM1, STAGES>;
   auto kern = mx_grouped_gemm_kernel<GEMM1, STAGES>;
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
-  return launch_k(kern, dim3(num_sms()), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, args);
+  return launch_k(kern, dim3(num_sms()), dim3(Cf::THREADS), Cf::ALLOC, stream, a, b, c, args);
 }
 
 }  // namespace
@@ -573,7 +616,7 @@ cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint3
   if (use_mx_swap(p.R, p.E))
     return launch_gemm1_mx_swap(p, xq, sxw, row2assign, offsets, w13p, w13sf, act, act_sf,
                                 act_sfw, status, stream, launches);
-  CUtensorMap ta{}, tb;
+  CUtensorMap ta{}, tb, tc{};
   if (!make_tmap_fp4(&tb, w13p, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, 128))
     return cudaErrorInvalidValue;
   MxArgs a{};
@@ -596,7 +639,7 @@ cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint3
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mx<true, 4>(ta, tb, a, stream);
+  return run_mx<true, 4>(ta, tb, tc, a, stream);
 }
 
 cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint32_t* act_sfw,
@@ -605,9 +648,10 @@ cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint
   if (p.R == 0) return cudaSuccess;
   if (use_mx_swap(p.R, p.E))
     return launch_gemm2_mx_swap(p, act, act_sfw, offsets, w2p, w2sf, y, status, stream, launches);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap_u8(&ta, act, p.I, p.R, BM) ||
-      !make_tmap_fp4(&tb, w2p, p.I, static_cast<uint64_t>(p.E) * p.H, 128))
+      !make_tmap_fp4(&tb, w2p, p.I, static_cast<uint64_t>(p.E) * p.H, 128) ||
+      !make_tmap_epi(encode_fn_mx(), &tc, y, p.H, p.R))
     return cudaErrorInvalidValue;
   MxArgs a{};
   a.offsets = offsets;
@@ -625,7 +669,7 @@ cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mx<false, 6>(ta, tb, a, stream);
+  return run_mx<false, 6>(ta, tb, tc, a, stream);
 }
 
 }  // namespace moe

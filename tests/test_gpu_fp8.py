@@ -66,6 +66,9 @@ SMALL = {
     "e512_k10_t7": I.Workload("s2", 7, 256, 256, 512, 10, dtype="fp8_mxfp4", routing="uniform"),
     "ragged_t129_h384": I.Workload("s3", 129, 384, 256, 4, 2, dtype="fp8_mxfp4"),
     "fp8_shape_t64": W["fp8_mxfp4"].with_T(64),
+    # > 48 rows per expert: the single-SM block-scaled kernels, 5 and 8 K blocks in GEMM2
+    "e8_t300_i640": I.Workload("s4", 300, 256, 640, 8, 2, dtype="fp8_mxfp4"),
+    "e4_t200_i1024": I.Workload("s5", 200, 256, 1024, 4, 2, dtype="fp8_mxfp4"),
 }
 
 

@@ -12,6 +12,8 @@
 //
 // Weight preparation: FlashInfer PR #6465, MXFP4 weights with K32 UE8M0 scaling; the
 // scale follows the OCP MX rule 2^(floor(log2 amax) - 2).
+#include <algorithm>
+
 #include "kernels.h"
 #include "launch.cuh"
 #include "sm100.cuh"
@@ -97,32 +99,49 @@ __global__ void __launch_bounds__(kCombineThreads)
   }
 }
 
-// One warp per (token, 128-column group); each lane owns 4 consecutive columns.
+// Two (token, 128-column group)s per warp iteration, one per half-warp; each lane owns 8
+// consecutive columns (one 16-byte load, one 8-byte store).  Warps stride over the groups
+// so that a few thousand CTAs cover any T.
 __global__ void __launch_bounds__(256)
     quant_x_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ xq,
                    float* __restrict__ sx, uint32_t* __restrict__ sxw, int64_t groups, int H) {
   const int lane = threadIdx.x & 31;
-  const int64_t gid = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int hl = lane & 15;
   pdl_wait();
   pdl_launch_dependents();
-  if (gid >= groups) return;
   const int G = H / 128;
-  const int64_t t = gid / G;
-  const int g = static_cast<int>(gid % G);
-  const int64_t base = t * H + g * 128 + lane * 4;
-  const uint2 v = __ldg(reinterpret_cast<const uint2*>(x + base));
-  const float f0 = bf16_lo(v.x), f1 = bf16_hi(v.x), f2 = bf16_lo(v.y), f3 = bf16_hi(v.y);
-  float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); w * 2 < groups;
+       w += nwarps) {  // warp-uniform condition: both halves stay in the loop together
+    const int64_t gid = w * 2 + (lane >> 4);
+    const bool ok = gid < groups;
+    const int64_t t = gid / G;
+    const int g = static_cast<int>(gid - t * G);
+    const int64_t base = t * H + g * 128 + hl * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) v = __ldg(reinterpret_cast<const uint4*>(x + base));
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.0f;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const int s = fp8_scale_exponent(amax);
-  const float inv = pow2f(-s);
-  const uint32_t lo = cvt_e4m3x2(f0 * inv, f1 * inv);
-  const uint32_t hi = cvt_e4m3x2(f2 * inv, f3 * inv);
-  *reinterpret_cast<uint32_t*>(xq + base) = lo | (hi << 16);
-  if (lane == 0) {
-    sx[t * G + g] = pow2f(s);
-    if (sxw) sxw[t * G + g] = static_cast<uint32_t>(s + 127) * 0x01010101u;
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1)  // within the half-warp
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int sc = fp8_scale_exponent(amax);
+    const float inv = pow2f(-sc);
+    uint2 q;
+    q.x = static_cast<uint32_t>(cvt_e4m3x2(f[0] * inv, f[1] * inv)) |
+          (static_cast<uint32_t>(cvt_e4m3x2(f[2] * inv, f[3] * inv)) << 16);
+    q.y = static_cast<uint32_t>(cvt_e4m3x2(f[4] * inv, f[5] * inv)) |
+          (static_cast<uint32_t>(cvt_e4m3x2(f[6] * inv, f[7] * inv)) << 16);
+    if (ok) {
+      *reinterpret_cast<uint2*>(xq + base) = q;
+      if (hl == 0) {
+        sx[t * G + g] = pow2f(sc);
+        if (sxw) sxw[t * G + g] = static_cast<uint32_t>(sc + 127) * 0x01010101u;
+      }
+    }
   }
 }
 
@@ -197,8 +216,9 @@ cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* 
   const int64_t groups = T * (H / 128);
   if (groups == 0) return cudaSuccess;
   ++*launches;
-  return launch_k(quant_x_kernel, dim3(static_cast<unsigned>((groups + 7) / 8)), dim3(256), 0, stream,
-                  x, xq, sx, sxw, groups, H);
+  const int64_t blocks = std::min<int64_t>((groups + 15) / 16, 16 * num_sms());
+  return launch_k(quant_x_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, x, xq,
+                  sx, sxw, groups, H);
 }
 
 cudaError_t launch_quant_w_mxfp4(const uint16_t* w, uint8_t* packed, uint8_t* sf, int64_t rows,

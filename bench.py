@@ -43,8 +43,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # gemm_swap_decode_T1, gemm_mx_swap_fp8_mxfp4_T128); an entry is removed when its kernel
 # changes after the capture.
 NCU_TRAFFIC = {
-    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 968.32e6 + 92.68e6,
-    ("qwen3_30b_a3b", 8192, "gemm2"): 503.48e6 + 238.04e6,
+    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 968.51e6 + 94.64e6,
+    ("qwen3_30b_a3b", 8192, "gemm2"): 503.43e6 + 238.33e6,
     ("decode", 1, "gemm1_swiglu"): 469.82e6 + 4.16e6,
     ("decode", 1, "gemm2"): 234.98e6 + 3.68e6,
     ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.71e6 + 4.96e6,

@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
     tmem_relinquish();
   }
   pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  pdl_launch_dependents();  // the next kernel's CTAs may take SMs as this grid's CTAs exit
   for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {  // m-tile prefix over experts; lane l owns a contiguous expert range
@@ -420,7 +421,6 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
     epi_drain(lane);
   }
 
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -143,6 +143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
     tmem_relinquish_2sm();
   }
   pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  pdl_launch_dependents();  // the next kernel's CTAs may take SMs as this grid's CTAs exit
   for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {  // pair-tile prefix over experts (256 rows per pair tile)
@@ -411,7 +412,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<GEMM1, STAGE
     epi_drain(lane);
   }
 
-  pdl_launch_dependents();
   tc_fence_before();
   cluster_sync();  // neither CTA leaves while the pair's MMAs or signals may touch it
   if (warp == 1) {

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     tmem_relinquish();
   }
   pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  pdl_launch_dependents();  // the next kernel's CTAs may take SMs as this grid's CTAs exit
   for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {
@@ -518,7 +519,6 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
     if constexpr (!GEMM1) epi_drain(lane);
   }
 
-  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

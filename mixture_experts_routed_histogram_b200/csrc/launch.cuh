@@ -2,7 +2,10 @@
 // start on free SMs while its predecessor on the stream is finishing, runs its prologue
 // (barrier init, TMEM allocation, tensor-map prefetch), and waits in pdl_wait() until the
 // predecessor has completed and its memory is visible before it touches any global data
-// the predecessor produces or reads.  MOE_PDL=0 turns the overlap off.
+// the predecessor produces or reads.  Every kernel signals pdl_launch_dependents() right
+// after its own pdl_wait(): the successor's CTAs are then scheduled as soon as SM resources
+// free up (the persistent GEMMs' tail wave), which is safe because the successor's
+// pdl_wait() still waits for this grid's completion.  MOE_PDL=0 turns the overlap off.
 #pragma once
 
 #include <cuda_runtime.h>

@@ -1,7 +1,12 @@
 """Failure detection without a GPU fault: a test hook leaves one pipeline stage of a
 grouped-GEMM launch unfilled, the consumer's bounded mbarrier wait (shortened to 50 ms)
 expires, every role of the kernel unwinds, the status word reads MOE_ERR_DEVICE_TIMEOUT,
-and the context stays usable: the next launches give correct results."""
+and the context stays usable: the same launch without the hook gives the same bits as a
+clean launch made before the failure (and the first case also matches the oracle).
+
+The shapes pick each GEMM kernel family: decode-sized (weights on the MMA's M side),
+single-SM tiles, SM-pair tiles (GEMM2 at >= 768 rows per expert), and the block-scaled
+FP8 x MXFP4 kernels in both their forms."""
 import numpy as np
 import pytest
 import torch
@@ -13,55 +18,85 @@ from mixture_experts_routed_histogram_b200 import inputs as I
 
 pytestmark = pytest.mark.gpu
 
+CASES = {
+    "bf16_swap": I.WORKLOADS["tiny"],                                  # T <= 64
+    "bf16_single_sm": I.Workload("fs", 300, 256, 128, 8, 2),           # 75 rows / expert
+    "bf16_pair_gemm2": I.Workload("fp", 2048, 256, 128, 2, 1),         # 1024 rows / expert
+    "fp8_single_sm": I.Workload("f8", 300, 256, 256, 4, 2, dtype="fp8_mxfp4"),
+    "fp8_swap": I.Workload("f8s", 64, 256, 128, 8, 2, dtype="fp8_mxfp4"),
+}
 
-def _case():
-    wl = I.WORKLOADS["tiny"]
+
+def _setup(wl):
     inp = I.make_inputs(wl, 0, dev())
     oids, _ = oracle_route(wl, inp["logits"])
     _, oo, or2a, _ = oracle.permute(oids, wl.E)
-    return wl, inp, oo, or2a
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    fp8 = wl.dtype == "fp8_mxfp4"
+    st = {"inp": inp, "oo": oo, "or2a": or2a, "shape": shape, "ws": ws, "fp8": fp8}
+    if fp8:
+        xq = torch.empty(wl.T, wl.H, dtype=torch.uint8, device=dev())
+        sx = torch.empty(wl.T, wl.H // 128, dtype=torch.float32, device=dev())
+        C.moe_quantize_x(shape, inp["x"], xq, sx)
+        rng = np.random.default_rng(5)
+        aq, sa = oracle.quant_fp8(rng.standard_normal((wl.R, wl.I)))
+        st.update(xq=xq, sx=sx, a_in=torch.from_numpy(aq).to(dev()),
+                  sa_in=torch.from_numpy(sa).to(dev()))
+    else:
+        g = torch.Generator(device=dev()).manual_seed(3)
+        st["a_in"] = torch.randn(wl.R, wl.I, generator=g, device=dev()).to(torch.bfloat16)
+        st["sa_in"] = None
+    return st
 
 
-def _gemm1(shape, wl, inp, oo, or2a, ws):
-    act = torch.empty(wl.R, wl.I, dtype=torch.bfloat16, device=dev())
-    C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, to_dev_i32(or2a), to_dev_i32(oo),
-                               inp["w13"], None, act, None, ws)
-    return act
-
-
-def _gemm2(shape, wl, inp, oo, act, ws):
+def _run(wl, st, which):
+    inp, shape, ws = st["inp"], st["shape"], st["ws"]
+    if which == "gemm1":
+        if st["fp8"]:
+            act = torch.empty(wl.R, wl.I, dtype=torch.uint8, device=dev())
+            act_sf = torch.empty(wl.R, wl.I // 128, dtype=torch.float32, device=dev())
+            C.moe_grouped_gemm1_swiglu(shape, st["xq"], st["sx"], to_dev_i32(st["or2a"]),
+                                       to_dev_i32(st["oo"]), inp["w13"], inp["w13_sf"], act,
+                                       act_sf, ws)
+            return torch.cat([act.view(-1), act_sf.view(torch.uint8).view(-1)])
+        act = torch.empty(wl.R, wl.I, dtype=torch.bfloat16, device=dev())
+        C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, to_dev_i32(st["or2a"]),
+                                   to_dev_i32(st["oo"]), inp["w13"], None, act, None, ws)
+        return act
     y = torch.empty(wl.R, wl.H, dtype=torch.bfloat16, device=dev())
-    C.moe_grouped_gemm2(shape, act, None, to_dev_i32(oo), inp["w2"], None, y, ws)
+    C.moe_grouped_gemm2(shape, st["a_in"], st["sa_in"], to_dev_i32(st["oo"]), inp["w2"],
+                        inp.get("w2_sf"), y, ws)
     return y
 
 
 @pytest.mark.parametrize("which", ["gemm1", "gemm2"])
-def test_injected_stall_reports_timeout_and_context_survives(which):
-    wl, inp, oo, or2a = _case()
-    shape = C.MoeShape.from_workload(wl)
-    ws = workspace(shape)
-    g = torch.Generator(device=dev()).manual_seed(3)
-    act_in = torch.randn(wl.R, wl.I, generator=g, device=dev()).to(torch.bfloat16)
+@pytest.mark.parametrize("case", list(CASES))
+def test_injected_stall_reports_timeout_and_context_survives(case, which):
+    wl = CASES[case]
+    st = _setup(wl)
+    clean = _run(wl, st, which).clone()
+    torch.cuda.synchronize()
+    assert C.moe_get_device_status(st["ws"]) == 0
     C.moe_debug_set_wait_limit_ns(50_000_000)
     C.moe_debug_inject_stall(True)
     try:
-        if which == "gemm1":
-            _gemm1(shape, wl, inp, oo, or2a, ws)
-        else:
-            _gemm2(shape, wl, inp, oo, act_in, ws)
+        _run(wl, st, which)
         torch.cuda.synchronize()
-        assert C.moe_get_device_status(ws) == C.MOE_ERR_DEVICE_TIMEOUT
+        assert C.moe_get_device_status(st["ws"]) == C.MOE_ERR_DEVICE_TIMEOUT
     finally:
         C.moe_debug_inject_stall(False)
         C.moe_debug_set_wait_limit_ns(0)
-    # the same launch again, without the hook: correct, and no status
-    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
-    if which == "gemm1":
-        out = _gemm1(shape, wl, inp, oo, or2a, ws)
-        ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), or2a // wl.k, ex)
-    else:
-        out = _gemm2(shape, wl, inp, oo, act_in, ws)
-        ref = oracle.gemm2_bf16_rows(I.bits(act_in), I.bits(inp["w2"]), np.arange(wl.R), ex)
+    again = _run(wl, st, which)
     torch.cuda.synchronize()
-    assert C.moe_get_device_status(ws) == 0
-    assert_close(f64(out), ref, what=f"{which} after recovery")
+    assert C.moe_get_device_status(st["ws"]) == 0
+    assert torch.equal(again.view(torch.uint8), clean.view(torch.uint8)), "results changed"
+    if case == "bf16_swap":   # and the clean result is the oracle's
+        inp, oo, or2a = st["inp"], st["oo"], st["or2a"]
+        ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+        if which == "gemm1":
+            ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), or2a // wl.k, ex)
+        else:
+            ref = oracle.gemm2_bf16_rows(I.bits(st["a_in"]), I.bits(inp["w2"]),
+                                         np.arange(wl.R), ex)
+        assert_close(f64(again), ref, what=f"{which} after recovery")

@@ -60,11 +60,13 @@ struct MxArgs {
   uint64_t wait_limit_ns;
 };
 
-template <bool GEMM1, int STAGES>
+// GEMM2 runs with BN2 = 256 (one accumulator, handed back right after the epilogue has
+// read it) when H % 256 == 0, else with BN2 = 128 (two accumulators).
+template <bool GEMM1, int BN2, int STAGES>
 struct MxCfg {
-  static constexpr int BN = GEMM1 ? 256 : 128;       // MMA N
-  static constexpr int BN_OUT = GEMM1 ? 128 : 128;   // output columns per tile
-  static constexpr int NACC = GEMM1 ? 1 : 2;         // TMEM accumulators
+  static constexpr int BN = GEMM1 ? 256 : BN2;       // MMA N
+  static constexpr int BN_OUT = GEMM1 ? 128 : BN2;   // output columns per tile
+  static constexpr int NACC = BN == 256 ? 1 : 2;     // TMEM accumulators
   static constexpr int THREADS = GEMM1 ? 32 * (6 + kLoaderWarps) : 32 * 7;
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;            // shared-memory footprint
@@ -115,12 +117,12 @@ __device__ __forceinline__ float silu_mul_mx(float g, float u) {
 // byte offset of row r (0..127) in a 512-byte scale atom
 __device__ __forceinline__ int sf_atom_off(int r) { return 16 * (r & 31) + 4 * (r >> 5); }
 
-template <bool GEMM1, int STAGES>
-__global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
+template <bool GEMM1, int BN2, int STAGES>
+__global__ void __launch_bounds__(MxCfg<GEMM1, BN2, STAGES>::THREADS, 1)
     mx_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmC, const MxArgs args) {
-  using C = MxCfg<GEMM1, STAGES>;
+  using C = MxCfg<GEMM1, BN2, STAGES>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -230,7 +232,9 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
           } else {
             mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_TX);
             tma_load_2d(a_dst, &tmA, &full[s], kb * BK, row0);
-            tma_load_2d(b_dst, &tmB, &full[s], kb * BK, brow);
+#pragma unroll
+            for (int b = 0; b < BN / 128; ++b)
+              tma_load_2d(b_dst + b * 128 * BK, &tmB, &full[s], kb * BK, brow + 128 * b);
           }
         }
         __syncwarp();
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
         }
       }
     } else {
-      // one warp: the stage's scale atoms (128 A rows, 128 B rows) -- 8 words per lane
+      // one warp: the stage's scale atoms (128 A rows, BN B rows) -- 4 + BN/32 words per lane
       const int G = args.K / 128;
       for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
         int e, mt, nt;
@@ -390,14 +394,16 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
         const int64_t row0 = s_off[e] + mt * BM;
         const int64_t brow = static_cast<int64_t>(e) * args.b_rows + nt * C::BN_OUT;
         const uint32_t* sfa_src[4];
-        const uint8_t* sfb_src[4];
+        const uint8_t* sfb_src[BN / 32];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int r = lane + 32 * j;
           const int64_t ra = min(row0 + r, args.R - 1);  // rows past the end: any valid row
           sfa_src[j] = args.a_sfw + ra * G;
-          sfb_src[j] = args.b_sf + (brow + r) * sf_row_bytes;
         }
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j)
+          sfb_src[j] = args.b_sf + (brow + lane + 32 * j) * sf_row_bytes;
         for (int kb = 0; kb < kblocks; ++kb, ++fill) {
           const int s = fill % STAGES;
           const uint32_t ph = (fill / STAGES) & 1u;
@@ -407,11 +413,12 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
           }
           const uint32_t sf_base = smem_u32(smem + C::SF_OFF + s * C::SF_BYTES);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int off = 16 * lane + 4 * j;  // row lane + 32 j
-            cp_async_4(sf_base + off, sfa_src[j] + kb);
-            cp_async_4(sf_base + 512 + off, sfb_src[j] + kb * 4);
-          }
+          for (int j = 0; j < 4; ++j)  // row lane + 32 j of the atom
+            cp_async_4(sf_base + 16 * lane + 4 * j, sfa_src[j] + kb);
+#pragma unroll
+          for (int j = 0; j < BN / 32; ++j)  // B row lane + 32 j: atom j / 4, slot j % 4
+            cp_async_4(sf_base + 512 + 512 * (j >> 2) + 16 * lane + 4 * (j & 3),
+                       sfb_src[j] + kb * 4);
           cp_async_mbar_arrive_noinc(&full[s]);
         }
       }
@@ -486,6 +493,36 @@ __global__ void __launch_bounds__(MxCfg<GEMM1, STAGES>::THREADS, 1)
           const int64_t gi = row * (args.n_out / 128) + nt;
           if (args.out_sf) args.out_sf[gi] = pow2f(se);
           args.out_sfw[gi] = static_cast<uint32_t>(se + 127) * 0x01010101u;
+        }
+      } else if constexpr (C::NACC == 1) {
+        // single accumulator: read all BN columns as packed bf16 pairs, hand the
+        // accumulator back to the MMA warp, then stage and store
+        uint16_t* y = static_cast<uint16_t*>(args.out);
+        uint32_t pk[BN / 32][16];
+#pragma unroll
+        for (int c = 0; c < BN / 32; c += 2) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(tb + 32 * c, v0);
+          tmem_ld_32x32b_x32(tb + 32 * c + 32, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pk[c][i] = pack_bf16x2(__uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+            pk[c + 1][i] = pack_bf16x2(__uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col = nt * C::BN_OUT + 32 * c;
+          if (col < args.n_out) {
+            if (whole)
+              epi_store_chunk(st, &tmC, pk[c], col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(y + row * args.n_out + col, pk[c]);
+          }
         }
       } else {
         uint16_t* y = static_cast<uint16_t*>(args.out);
@@ -586,11 +623,11 @@ bool make_tmap_fp4(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GEMM1, int STAGES>
+template <bool GEMM1, int BN2, int STAGES>
 cudaError_t run_mx(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                    const MxArgs& args, cudaStream_t stream) {
-  using Cf = MxCfg<GEMM1, STAGES>;
-  auto kern = mx_grouped_gemm_kernel<GEMM1, STAGES>;
+  using Cf = MxCfg<GEMM1, BN2, STAGES>;
+  auto kern = mx_grouped_gemm_kernel<GEMM1, BN2, STAGES>;
   static cudaError_t attr =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::ALLOC);
   if (attr != cudaSuccess) return attr;
@@ -639,7 +676,7 @@ cudaError_t launch_gemm1_mx(const GemmProblem& p, const uint8_t* xq, const uint3
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mx<true, 4>(ta, tb, tc, a, stream);
+  return run_mx<true, 256, 4>(ta, tb, tc, a, stream);
 }
 
 cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint32_t* act_sfw,
@@ -663,13 +700,15 @@ cudaError_t launch_gemm2_mx(const GemmProblem& p, const uint8_t* act, const uint
   a.k_top = p.k;
   a.n_out = p.H;
   a.K = p.I;
-  a.n_tiles = p.H / 128;
+  const bool wide = p.H % 256 == 0;
+  a.n_tiles = p.H / (wide ? 256 : 128);
   a.b_rows = p.H;
   a.R = p.R;
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
-  return run_mx<false, 6>(ta, tb, tc, a, stream);
+  return wide ? run_mx<false, 256, 4>(ta, tb, tc, a, stream)
+              : run_mx<false, 128, 6>(ta, tb, tc, a, stream);
 }
 
 }  // namespace moe

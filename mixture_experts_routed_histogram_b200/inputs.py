@@ -14,6 +14,10 @@ Workloads (shapes and value recipes):
                   renormalised, uniform expert load (FlashInfer PR #6465 workload).
   decode          T in {1, 8, 32, 128, 256}, H=4096, E=8, k=2, I=14336, softmax top-2
                   renormalised, Zipf(1.2)-skewed expert choice with one expert never chosen.
+  grid_d{D}_e{E}_k{k}
+                  the parameter grid of the Liger-Kernel PR #1463 benchmark: T=8192,
+                  H=I=D in {2048, 4096}, E in {8, 16, 32, 64, 128}, k in {1, 2, 4, 8} with
+                  k < E (38 shapes), softmax top-k renormalised, gaussian routing.
 
 Values: x ~ N(0,1) bf16; W13 ~ N(0, 1/H) and W2 ~ N(0, 1/I) bf16 (fan-in scaling).
 Router logits:
@@ -69,6 +73,9 @@ WORKLOADS = {
                           routing="uniform"),
     "decode": Workload("decode", 32, 4096, 14336, 8, 2, routing="zipf"),
 }
+GRID = {f"grid_d{d}_e{e}_k{k}": Workload(f"grid_d{d}_e{e}_k{k}", 8192, d, d, e, k)
+        for d in (2048, 4096) for e in (8, 16, 32, 64, 128) for k in (1, 2, 4, 8) if k < e}
+WORKLOADS.update(GRID)
 FP8_T_SWEEP = (128, 1024, 8192, 16384)
 DECODE_T_SWEEP = (1, 8, 32, 128, 256)
 

@@ -68,8 +68,13 @@ def lib():
             L.orc_forward_fp8_mxfp4.argtypes = [i64, i32, i32, i32, i32, _P(u16), _P(ctypes.c_int32),
                                                 _P(f64), _P(u8), _P(u8), _P(u8), _P(u8), i32, i64,
                                                 _P(i64), _P(f64), _P(u16)]
+            L.orc_forward_bf16_act.argtypes = [i64, i32, i32, i32, i32, i32, _P(u16),
+                                               _P(ctypes.c_int32), _P(f64), _P(u16), _P(u16),
+                                               i64, _P(i64), _P(f64), _P(u16)]
             L.orc_gemm1_bf16_rows.argtypes = [i32, i32, _P(u16), _P(u16), i64, _P(i64),
                                               _P(ctypes.c_int32), _P(f64)]
+            L.orc_gemm1_bf16_rows_act.argtypes = [i32, i32, i32, _P(u16), _P(u16), i64, _P(i64),
+                                                  _P(ctypes.c_int32), _P(f64)]
             L.orc_gemm2_bf16_rows.argtypes = [i32, i32, _P(u16), _P(u16), i64, _P(i64),
                                               _P(ctypes.c_int32), _P(f64)]
             L.orc_gemm1_fp8_rows.argtypes = [i32, i32, _P(u8), _P(f32), _P(u8), _P(u8), i32, i64,
@@ -234,22 +239,26 @@ def _toklist(tokens, T):
     return _c(tokens, np.int64)
 
 
-def forward_bf16(x_bits, ids, w, w13_bits, w2_bits, tokens=None):
-    """out[n] = sum_j w[t,j] * (silu(x_t.Wg^T) * (x_t.Wu^T)).Wd^T for t = tokens[n]."""
+ACTS = {"swiglu": 0, "relu2": 1}
+
+
+def forward_bf16(x_bits, ids, w, w13_bits, w2_bits, tokens=None, act="swiglu"):
+    """out[n] = sum_j w[t,j] * act_e(x_t).Wd^T for t = tokens[n], with act_e =
+    silu(x.Wg^T) * (x.Wu^T) (W13 [E, 2I, H]) or max(x.W1^T, 0)^2 (relu2, W1 [E, I, H])."""
     x = _c(x_bits, np.uint16); ids = _c(ids, np.int32); w = _c(w, np.float64)
     w13 = _c(w13_bits, np.uint16); w2 = _c(w2_bits, np.uint16)
     T, H = x.shape
-    E, twoI, H2 = w13.shape
-    assert H2 == H and w2.shape == (E, H, twoI // 2)
-    I = twoI // 2
+    E, rows, H2 = w13.shape
+    I = rows if act == "relu2" else rows // 2
+    assert H2 == H and w2.shape == (E, H, I)
     k = ids.shape[1]
     tok = _toklist(tokens, T)
     out = np.empty((len(tok), H), np.float64)
     ob = np.empty((len(tok), H), np.uint16)
-    lib().orc_forward_bf16(T, H, I, E, k, _ptr(x, np.uint16), _ptr(ids, np.int32),
-                           _ptr(w, np.float64), _ptr(w13, np.uint16), _ptr(w2, np.uint16),
-                           len(tok), _ptr(tok, np.int64), _ptr(out, np.float64),
-                           _ptr(ob, np.uint16))
+    lib().orc_forward_bf16_act(T, H, I, E, k, ACTS[act], _ptr(x, np.uint16),
+                               _ptr(ids, np.int32), _ptr(w, np.float64), _ptr(w13, np.uint16),
+                               _ptr(w2, np.uint16), len(tok), _ptr(tok, np.int64),
+                               _ptr(out, np.float64), _ptr(ob, np.uint16))
     return out, ob
 
 
@@ -276,14 +285,15 @@ def forward_fp8_mxfp4(x_bits, ids, w, w13p, w13sf, w2p, w2sf, tokens=None, requa
     return out, ob
 
 
-def gemm1_bf16_rows(x_bits, w13_bits, tok, expert):
+def gemm1_bf16_rows(x_bits, w13_bits, tok, expert, act="swiglu"):
     x = _c(x_bits, np.uint16); w13 = _c(w13_bits, np.uint16)
     tok = _c(tok, np.int64); ex = _c(expert, np.int32)
-    H = x.shape[1]; I = w13.shape[1] // 2
-    act = np.empty((len(tok), I), np.float64)
-    lib().orc_gemm1_bf16_rows(H, I, _ptr(x, np.uint16), _ptr(w13, np.uint16), len(tok),
-                              _ptr(tok, np.int64), _ptr(ex, np.int32), _ptr(act, np.float64))
-    return act
+    H = x.shape[1]; I = w13.shape[1] if act == "relu2" else w13.shape[1] // 2
+    out = np.empty((len(tok), I), np.float64)
+    lib().orc_gemm1_bf16_rows_act(ACTS[act], H, I, _ptr(x, np.uint16), _ptr(w13, np.uint16),
+                                  len(tok), _ptr(tok, np.int64), _ptr(ex, np.int32),
+                                  _ptr(out, np.float64))
+    return out
 
 
 def gemm2_bf16_rows(a_bits, w2_bits, rows, expert):

@@ -21,6 +21,9 @@
  *   expert MLP   g = h.Wgate^T, u = h.Wup^T, a = silu(g)*u, y = a.Wdown^T
  *                (TileScale PR #70, "Design": kernel 1 is GEMM1 + SwiGLU, kernel 2 is
  *                GEMM2).  Gate rows come first in the fused [2I, H] matrix (reading).
+ *                The ReLU2 variant (FlashInfer PR #5129, the Nemotron-3.5-Lightning
+ *                shape measured with ReLU2): g = h.W1^T with W1 [I, H], a = max(g, 0)^2
+ *                -- read as the non-gated squared ReLU, the pages name only "ReLU2".
  *   combine      out[t] = sum over slots j (ascending) of w[t,j] * y_j, rounded once to
  *                bf16 (TileScale PR #70, the top-k slot reduction of kernel 2).
  *   block-scaled activations: FP8 e4m3 with one power-of-two fp32 scale per 1x128 group
@@ -294,6 +297,26 @@ static void expert_act_bf16(int H, int I, const double *h, const uint16_t *w13e,
   }
 }
 
+/* act[i] = max(h . W1[i], 0)^2; W1 is this expert's [I, H] bf16 block (ReLU2). */
+static void expert_act_relu2_bf16(int H, int I, const double *h, const uint16_t *w1e,
+                                  double *act) {
+  for (int i = 0; i < I; ++i) {
+    double g = 0.0;
+    const uint16_t *wr = w1e + (int64_t)i * H;
+    for (int c = 0; c < H; ++c) g += h[c] * orc_bf16_to_f64(wr[c]);
+    act[i] = g > 0.0 ? g * g : 0.0;
+  }
+}
+
+/* The activation of GEMM1: kind 0 = SwiGLU (W13 block [2I, H]), 1 = ReLU2 (W1 [I, H]). */
+static void expert_act_kind_bf16(int kind, int H, int I, const double *h,
+                                 const uint16_t *w13, int e, double *act) {
+  if (kind == 1)
+    expert_act_relu2_bf16(H, I, h, w13 + (int64_t)e * I * H, act);
+  else
+    expert_act_bf16(H, I, h, w13 + (int64_t)e * 2 * I * H, act);
+}
+
 /* y[o] = act . W2[o]; W2 is this expert's [H, I] bf16 block. */
 static void expert_down_bf16(int H, int I, const double *act, const uint16_t *w2e, double *y) {
   for (int o = 0; o < H; ++o) {
@@ -340,10 +363,10 @@ static void requant_row_inplace(int I, double *act, uint8_t *codes, float *scale
 
 /* BF16 path.  ids/w come from orc_route.  For each listed token t:
  *   out[n][:] = sum_j w[t,j] * expert_mlp(ids[t,j], x[t]),  fp64, and its bf16 rounding. */
-void orc_forward_bf16(int64_t T, int H, int I, int E, int k, const uint16_t *x,
-                      const int32_t *ids, const double *w, const uint16_t *w13,
-                      const uint16_t *w2, int64_t n_tok, const int64_t *tok, double *out,
-                      uint16_t *out_bf16) {
+void orc_forward_bf16_act(int64_t T, int H, int I, int E, int k, int kind,
+                          const uint16_t *x, const int32_t *ids, const double *w,
+                          const uint16_t *w13, const uint16_t *w2, int64_t n_tok,
+                          const int64_t *tok, double *out, uint16_t *out_bf16) {
   (void)T; (void)E;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t n = 0; n < n_tok; ++n) {
@@ -355,13 +378,20 @@ void orc_forward_bf16(int64_t T, int H, int I, int E, int k, const uint16_t *x,
     for (int c = 0; c < H; ++c) { h[c] = orc_bf16_to_f64(x[t * H + c]); acc[c] = 0.0; }
     for (int j = 0; j < k; ++j) {
       int e = ids[t * k + j];
-      expert_act_bf16(H, I, h, w13 + (int64_t)e * 2 * I * H, act);
+      expert_act_kind_bf16(kind, H, I, h, w13, e, act);
       expert_down_bf16(H, I, act, w2 + (int64_t)e * H * I, y);
       for (int c = 0; c < H; ++c) acc[c] += w[t * k + j] * y[c];
     }
     for (int c = 0; c < H; ++c) out_bf16[n * H + c] = orc_f64_to_bf16_rne(acc[c]);
     free(h); free(act); free(y);
   }
+}
+
+void orc_forward_bf16(int64_t T, int H, int I, int E, int k, const uint16_t *x,
+                      const int32_t *ids, const double *w, const uint16_t *w13,
+                      const uint16_t *w2, int64_t n_tok, const int64_t *tok, double *out,
+                      uint16_t *out_bf16) {
+  orc_forward_bf16_act(T, H, I, E, k, 0, x, ids, w, w13, w2, n_tok, tok, out, out_bf16);
 }
 
 /* Block-scaled path: x is quantised per token (1x128 e4m3 + pow2 scale) and
@@ -402,16 +432,22 @@ void orc_forward_fp8_mxfp4(int64_t T, int H, int I, int E, int k, const uint16_t
 /* single stages on listed rows of the expert-sorted row space                          */
 /* ------------------------------------------------------------------------------------ */
 
-/* GEMM1 + SwiGLU for listed rows: row n uses token tok[n] of x and expert exp_[n]. */
-void orc_gemm1_bf16_rows(int H, int I, const uint16_t *x, const uint16_t *w13, int64_t n_rows,
-                         const int64_t *tok, const int32_t *exp_, double *act) {
+/* GEMM1 + activation for listed rows: row n uses token tok[n] of x and expert exp_[n]. */
+void orc_gemm1_bf16_rows_act(int kind, int H, int I, const uint16_t *x, const uint16_t *w13,
+                             int64_t n_rows, const int64_t *tok, const int32_t *exp_,
+                             double *act) {
 #pragma omp parallel for schedule(dynamic, 4)
   for (int64_t n = 0; n < n_rows; ++n) {
     double *h = (double *)malloc(sizeof(double) * (size_t)H);
     for (int c = 0; c < H; ++c) h[c] = orc_bf16_to_f64(x[tok[n] * H + c]);
-    expert_act_bf16(H, I, h, w13 + (int64_t)exp_[n] * 2 * I * H, act + n * I);
+    expert_act_kind_bf16(kind, H, I, h, w13, exp_[n], act + n * I);
     free(h);
   }
+}
+
+void orc_gemm1_bf16_rows(int H, int I, const uint16_t *x, const uint16_t *w13, int64_t n_rows,
+                         const int64_t *tok, const int32_t *exp_, double *act) {
+  orc_gemm1_bf16_rows_act(0, H, I, x, w13, n_rows, tok, exp_, act);
 }
 
 /* GEMM2 for listed rows: y[n] = a[row[n]] . W2[exp_[n]]^T with a given as bf16 rows. */

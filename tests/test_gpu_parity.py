@@ -230,6 +230,9 @@ FULL = {
     "qwen3_30b_a3b": W["qwen3_30b_a3b"],
     "llama4_scout": W["llama4_scout"],
     **{f"decode_T{t}": W["decode"].with_T(t) for t in I.DECODE_T_SWEEP},
+    # points of the parameter grid: 8192 rows per expert (top-1), 512 (E=128, top-8) and
+    # 2048 at H=I=4096 -- single-SM and SM-pair GEMM2, K up to 4096
+    **{n: W[n] for n in ("grid_d2048_e8_k1", "grid_d2048_e128_k8", "grid_d4096_e16_k4")},
 }
 
 

@@ -341,6 +341,63 @@ def test_forward_bf16_brute_force_tiny(orc, T, E, k, score):
     assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
 
 
+# ReLU2 variant (FlashInfer PR #5129, the Nemotron-3.5-Lightning shape): non-gated,
+# W1 [E, I, H], act = max(x.W1^T, 0)^2.
+
+def _relu2(g):
+    return np.where(g > 0, g * g, 0.0)
+
+
+def test_single_expert_top1_relu2_is_dense_squared_relu_mlp(orc):
+    rng = np.random.default_rng(22)
+    T, H, I = 9, 64, 48
+    xb = _rand_bf16(rng, (T, H))
+    w1 = _rand_bf16(rng, (1, I, H), H ** -0.5)
+    w2 = _rand_bf16(rng, (1, H, I), I ** -0.5)
+    ids = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1))
+    out, _ = orc.forward_bf16(xb, ids, w, w1, w2, act="relu2")
+    xv, g1, g2 = _bits_to_f64(xb), _bits_to_f64(w1)[0], _bits_to_f64(w2)[0]
+    dense = _relu2(xv @ g1.T) @ g2.T
+    assert np.allclose(out, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_relu2_hand_worked_rows(orc):
+    """h = (1, 2, -1, 0.5); rows of W1 chosen so that g = 3.5, -2, 0, 0.25 exactly:
+    act = 12.25, 0, 0, 0.0625; with W2 = ones, y = 12.3125 in every column."""
+    H, I = 4, 4
+    x = np.array([[1.0, 2.0, -1.0, 0.5]])
+    w1 = np.array([[[1, 1, 0, 1], [0, -1, 0, 0], [1, 0, 1, 0], [0, 0, 0, 0.5]]], float)
+    w2 = np.ones((1, H, I))
+    act = orc.gemm1_bf16_rows(_bf16_bits(x), _bf16_bits(w1), np.array([0]), np.array([0]),
+                              act="relu2")
+    assert np.array_equal(act[0], [12.25, 0.0, 0.0, 0.0625])
+    out, _ = orc.forward_bf16(_bf16_bits(x), np.zeros((1, 1), np.int32), np.ones((1, 1)),
+                              _bf16_bits(w1), _bf16_bits(w2), act="relu2")
+    assert np.array_equal(out[0], np.full(H, 12.3125))
+
+
+@pytest.mark.parametrize("T,E,k", [(8, 6, 2), (5, 4, 4), (3, 5, 1)])
+def test_forward_relu2_brute_force_tiny(orc, T, E, k):
+    rng = np.random.default_rng(T * 100 + E * 10 + k + 7)
+    H = I = 32
+    xb = _rand_bf16(rng, (T, H))
+    w1 = _rand_bf16(rng, (E, I, H), H ** -0.5)
+    w2 = _rand_bf16(rng, (E, H, I), I ** -0.5)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    ids, w = orc.route(lg, k)
+    out, _ = orc.forward_bf16(xb, ids, w, w1, w2, act="relu2")
+    xv, g1, g2 = _bits_to_f64(xb), _bits_to_f64(w1), _bits_to_f64(w2)
+    Y = np.stack([_relu2(xv @ g1[e].T) @ g2[e].T for e in range(E)])
+    sel = _topk_by_sort(lg, k)
+    ww = softmax(np.take_along_axis(lg.astype(np.float64), sel, 1), axis=1)
+    ref = np.zeros_like(xv)
+    for t in range(T):
+        for j in range(k):
+            ref[t] += ww[t, j] * Y[sel[t, j], t]
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
+
+
 def test_forward_token_subset_and_order_equivariance(orc):
     rng = np.random.default_rng(21)
     T, H, I, E, k = 12, 32, 32, 5, 2

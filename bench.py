@@ -222,17 +222,19 @@ def algorithmic(wl, counts):
     fp8 = wl.dtype == "fp8_mxfp4"
     wbytes = (0.5 + 1.0 / 32) if fp8 else 2.0     # per weight element (codes + scales)
     abytes = (1.0 + 4.0 / 128) if fp8 else 2.0     # per activation element (codes + scales)
-    f = {"gemm1_swiglu": 4.0 * R * H * Ii, "gemm2": 2.0 * R * H * Ii}
+    g1 = wl.gemm1_rows                              # 2I (SwiGLU) or I (ReLU2)
+    f = {"gemm1_swiglu": 2.0 * R * H * g1, "gemm2": 2.0 * R * H * Ii}
     b = {
         "route": T * E * 4 + R * 8,
         "permute": R * 4 * 3 + E * 8,
         "quantize_x": T * H * 2 + T * H * abytes,
-        "gemm1_swiglu": ne * 2 * Ii * H * wbytes + T * H * abytes + R * Ii * abytes + R * 4,
+        "gemm1_swiglu": ne * g1 * H * wbytes + T * H * abytes + R * Ii * abytes + R * 4,
         "gemm2": ne * H * Ii * wbytes + R * Ii * abytes + R * H * 2,
         "combine": R * H * 2 + T * H * 2 + R * 8,
     }
     # whole-pass bytes without the y round trip (a fused combine could avoid it)
-    b_alg = (ne * 3 * Ii * H * wbytes + T * H * 2 * 2 + R * Ii * abytes * 2 + T * E * 4 + R * 16)
+    b_alg = ((g1 + Ii) * ne * H * wbytes + T * H * 2 * 2 + R * Ii * abytes * 2 + T * E * 4
+             + R * 16)
     return f, b, b_alg, ne
 
 
@@ -439,7 +441,7 @@ def _oracle_forward(wl, x, ids, w, wts, toks):
     import oracle
     if wl.dtype == "fp8_mxfp4":
         return oracle.forward_fp8_mxfp4(x, ids, w, *wts, tokens=toks, requant_act=True)
-    return oracle.forward_bf16(x, ids, w, wts[0], wts[1], toks)
+    return oracle.forward_bf16(x, ids, w, wts[0], wts[1], toks, act=wl.act)
 
 
 def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
@@ -506,7 +508,7 @@ def bench_reference(args, rank, world):
         if s >= args.warmup:
             times.append(dt)
     sec = float(np.mean(times))
-    flops = 6.0 * n * wl.k * wl.H * wl.I
+    flops = 2.0 * n * wl.k * wl.H * (wl.gemm1_rows + wl.I)
     val = flops / sec / 1e12
     return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -70,15 +70,21 @@ typedef enum {
 
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
 typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_MXFP4 = 1 } moe_dtype_t;
+/* GEMM1's activation.  SWIGLU: W13 [E][2I][H] (gate rows then up rows), act =
+ * silu(gate) * up.  RELU2 (BF16 only; FlashInfer PR #5129 measures the Nemotron-3.5-
+ * Lightning shape with it, read as the non-gated squared ReLU): W13 is W1 [E][I][H] and
+ * act = max(x.W1^T, 0)^2. */
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act_t;
 
 /* Problem description.  score: moe_score_t; renormalize: 1 = divide the k selected
- * weights by their sum; dtype: moe_dtype_t. */
+ * weights by their sum; dtype: moe_dtype_t; activation: moe_act_t. */
 typedef struct {
   int64_t T;
   int32_t H, I, E, k;
   int32_t score;
   int32_t renormalize;
   int32_t dtype;
+  int32_t activation;
 } moe_shape_t;
 
 /* Bytes of device workspace moe_forward needs for `shape` (the stage entry points need
@@ -148,9 +154,10 @@ MOE_API moe_status_t moe_quantize_weights_mxfp4(int64_t rows, int32_t K, const u
 /* Grouped GEMM1 with fused SwiGLU over the expert-sorted rows (TileScale PR #70 kernel 1;
  * FlashInfer PR #5129 gathered-A GEMM1).  For sorted row r of expert e with token
  * t = row2assign[r] / k:  act[r][i] = silu(x[t].W13[e][i]) * (x[t].W13[e][I+i]), fp32
- * accumulation, silu(g) = g / (1 + exp(-g)).
- *   BF16:  a = x bf16 [T][H]; sa, w13_sf, act_sf unused (may be NULL); w13 bf16 [E][2I][H];
- *          act bf16 [R][I] out.
+ * accumulation, silu(g) = g / (1 + exp(-g)); with activation RELU2,
+ * act[r][i] = max(x[t].W1[e][i], 0)^2.
+ *   BF16:  a = x bf16 [T][H]; sa, w13_sf, act_sf unused (may be NULL); w13 bf16 [E][2I][H]
+ *          (RELU2: W1 bf16 [E][I][H]); act bf16 [R][I] out.
  *   FP8:   a = xq e4m3 [T][H]; sa = sx fp32 [T][H/128]; w13 = MXFP4 [E][2I][H/2];
  *          w13_sf = UE8M0 [E][2I][H/32]; act = e4m3 [R][I] out, requantised per 1x128
  *          with the moe_quantize_x rule; act_sf fp32 [R][I/128] out.

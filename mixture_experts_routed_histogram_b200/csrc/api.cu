@@ -61,8 +61,11 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E <= 0 || s->k <= 0) return MOE_ERR_INVALID_ARG;
   if ((s->score != MOE_SCORE_SOFTMAX && s->score != MOE_SCORE_SIGMOID) ||
       (s->dtype != MOE_DTYPE_BF16 && s->dtype != MOE_DTYPE_FP8_MXFP4) ||
-      (s->renormalize != 0 && s->renormalize != 1))
+      (s->renormalize != 0 && s->renormalize != 1) ||
+      (s->activation != MOE_ACT_SWIGLU && s->activation != MOE_ACT_RELU2))
     return MOE_ERR_INVALID_ARG;
+  if (s->activation == MOE_ACT_RELU2 && s->dtype != MOE_DTYPE_BF16)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s->k > s->E) return MOE_ERR_INVALID_ARG;
   if (s->k > moe::kMaxTopK || s->E > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s->T * static_cast<int64_t>(s->k) >= (static_cast<int64_t>(1) << 31))
@@ -96,6 +99,7 @@ moe::GemmProblem problem(const moe_shape_t& s) {
   p.I = s.I;
   p.E = s.E;
   p.k = s.k;
+  p.act = s.activation;
   p.wait_limit_ns = g_wait_limit_ns;
   return p;
 }
@@ -340,13 +344,16 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
       return MOE_ERR_CUDA;
   } else if (moe::use_swap_gemm(T) && shape->H % 128 == 0) {
     // decode-sized: weights on the MMA's M side; GEMM2 splits K and the combine adds the
-    // partial sums
+    // partial sums.  (GEMM1 with ReLU2 runs on the single-SM kernel.)
     const int splits = moe::swap_splits(p);
     float* part = at<float>(ws, L.part);  // GEMM1's partials are consumed before GEMM2's
-    if ((e = moe::launch_gemm1_swap(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
-                                    part, moe::swap_splits_gemm1(p), status, stream, &n)) !=
-        cudaSuccess)
-      return MOE_ERR_CUDA;
+    if (p.act == MOE_ACT_RELU2)
+      e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+                                 status, stream, &n);
+    else
+      e = moe::launch_gemm1_swap(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
+                                 part, moe::swap_splits_gemm1(p), status, stream, &n);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     if ((e = moe::launch_gemm2_swap(p, act, offsets, static_cast<const uint16_t*>(w2), y, part,
                                     splits, status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;

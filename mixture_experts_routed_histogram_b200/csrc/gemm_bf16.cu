@@ -110,7 +110,11 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <bool GEMM1, int AMODE, int BN, int STAGES>
+__device__ __forceinline__ float relu2(float g) { return g > 0.0f ? g * g : 0.0f; }
+
+// ACT (GEMM1): 0 = SwiGLU, the tile's B rows are BN/2 gate rows and the matching BN/2 up
+// rows and it outputs BN/2 columns; 1 = ReLU2, BN consecutive W1 rows, BN output columns.
+template <bool GEMM1, int AMODE, int BN, int STAGES, int ACT = 0>
 __global__ void __launch_bounds__(threads_for(AMODE), 1)
     grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
   using L = Layout<BN, STAGES>;
   constexpr int kThreads = threads_for(AMODE);
   static_assert(GEMM1 || AMODE == kATile, "GEMM2 reads contiguous rows");
-  constexpr int BN_OUT = GEMM1 ? BN / 2 : BN;
+  constexpr int BN_OUT = GEMM1 && ACT == 0 ? BN / 2 : BN;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32<BM, BN>();
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
@@ -240,7 +244,8 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
             tma_gather4(a_dst + lane * 4 * 128, &tmA, &full[s], kb * BK, tk0, tk1, tk2, tk3);
           if (lane == 0) {
             tma_load_2d(b_dst, &tmB, &full[s], kb * BK, brow);
-            tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[s], kb * BK, brow + args.n_out);
+            tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[s], kb * BK,
+                        brow + (ACT == 0 ? args.n_out : BN / 2));
           }
         } else {
           if (lane == 0) {
@@ -369,7 +374,26 @@ __global__ void __launch_bounds__(threads_for(AMODE), 1)
       const bool valid = r_in < rows;
       const bool whole = rows - q * 32 >= 32;  // all 32 rows of this warp are the expert's
       const int64_t row = row0 + r_in;
-      if constexpr (GEMM1) {
+      if constexpr (GEMM1 && ACT == 1) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v32[32];
+          tmem_ld_32x32b_x32(tb + c, v32);
+          tmem_ld_wait();
+          const int col = nt * BN_OUT + c;
+          if (col < args.n_out) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(relu2(__uint_as_float(v32[2 * i])),
+                                  relu2(__uint_as_float(v32[2 * i + 1])));
+            if (whole)
+              epi_store_chunk(st, &tmC, pk, col, row0 + q * 32, lane);
+            else if (valid)
+              epi_store_row(args.out + row * args.n_out + col, pk);
+          }
+        }
+      } else if constexpr (GEMM1) {
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           uint32_t g[32], u[32];
@@ -461,11 +485,11 @@ bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS;
 }
 
-template <bool GEMM1, int AMODE, int BN, int STAGES>
+template <bool GEMM1, int AMODE, int BN, int STAGES, int ACT = 0>
 cudaError_t run(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                 const KArgs& args, cudaStream_t stream) {
   using L = Layout<BN, STAGES>;
-  auto kern = grouped_gemm_bf16_kernel<GEMM1, AMODE, BN, STAGES>;
+  auto kern = grouped_gemm_bf16_kernel<GEMM1, AMODE, BN, STAGES, ACT>;
   static cudaError_t attr = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (attr != cudaSuccess) return attr;
@@ -500,17 +524,22 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
                               const int32_t* offsets, const uint16_t* w13, uint16_t* act,
                               int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
-  if (use_swap_gemm(p.T))
+  const bool relu2 = p.act == 1;
+  if (!relu2 && use_swap_gemm(p.T))
     return launch_gemm1_swap(p, x, row2assign, offsets, w13, act, nullptr, 1, status, stream,
                              launches);
-  if (p.I % 128 == 0 && !use_gather4() && use_pair_gemm1(p.R, p.E))
+  if (!relu2 && p.I % 128 == 0 && !use_gather4() && use_pair_gemm1(p.R, p.E))
     return launch_gemm1_bf16_2sm(p, x, row2assign, offsets, w13, act, status, stream, launches);
-  const bool wide = (p.I % 128) == 0;
+  // SwiGLU: 128 gate + 128 up rows per tile when I % 128 == 0, else 64 + 64;
+  // ReLU2: 256 consecutive W1 rows per tile (the last tile's columns past I are dropped)
+  const bool wide = relu2 || (p.I % 128) == 0;
   const int bn = wide ? 256 : 128;
+  const int bn_out = relu2 ? bn : bn / 2;
   CUtensorMap ta, tb;
   CUtensorMap tc;
   if (!make_tmap_bf16(&ta, x, p.H, p.T, BK, 1) ||
-      !make_tmap_bf16(&tb, w13, p.H, static_cast<uint64_t>(p.E) * 2 * p.I, BK, bn / 2) ||
+      !make_tmap_bf16(&tb, w13, p.H, static_cast<uint64_t>(p.E) * (relu2 ? 1 : 2) * p.I, BK,
+                      bn / 2) ||
       !make_tmap_epi(encode_fn(), &tc, act, p.I, p.R))
     return cudaErrorInvalidValue;
   KArgs a{};
@@ -523,11 +552,12 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   a.k_top = p.k;
   a.n_out = p.I;
   a.K = p.H;
-  a.n_tiles = (p.I + bn / 2 - 1) / (bn / 2);
-  a.b_rows = 2 * p.I;
+  a.n_tiles = (p.I + bn_out - 1) / bn_out;
+  a.b_rows = (relu2 ? 1 : 2) * p.I;
   a.inject_stall = g_inject_stall;
   a.wait_limit_ns = p.wait_limit_ns;
   ++*launches;
+  if (relu2) return run<true, kACpAsync, 256, 4, 1>(ta, tb, tc, a, stream);
   if (use_gather4())
     return wide ? run<true, kAGather4, 256, 4>(ta, tb, tc, a, stream)
                 : run<true, kAGather4, 128, 6>(ta, tb, tc, a, stream);

@@ -62,6 +62,7 @@ struct GemmProblem {
   int64_t T;      // tokens (GEMM1 A rows)
   int64_t R;      // routed rows
   int H, I, E, k;
+  int act;        // GEMM1 activation: 0 SwiGLU (W13 [E][2I][H]), 1 ReLU2 (W1 [E][I][H])
   uint64_t wait_limit_ns;
 };
 

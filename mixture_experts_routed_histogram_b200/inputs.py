@@ -14,6 +14,9 @@ Workloads (shapes and value recipes):
                   renormalised, uniform expert load (FlashInfer PR #6465 workload).
   decode          T in {1, 8, 32, 128, 256}, H=4096, E=8, k=2, I=14336, softmax top-2
                   renormalised, Zipf(1.2)-skewed expert choice with one expert never chosen.
+  nemotron_relu2  T=8192, H=2688, E=128, k=6, I=1856, ReLU2 (non-gated squared ReLU, W1
+                  [E, I, H]), softmax top-6 renormalised, gaussian routing: the
+                  Nemotron-3.5-Lightning shape FlashInfer PR #5129 measures.
   grid_d{D}_e{E}_k{k}
                   the parameter grid of the Liger-Kernel PR #1463 benchmark: T=8192,
                   H=I=D in {2048, 4096}, E in {8, 16, 32, 64, 128}, k in {1, 2, 4, 8} with
@@ -50,6 +53,7 @@ class Workload:
     renorm: bool = True
     dtype: str = "bf16"          # "bf16" | "fp8_mxfp4"
     routing: str = "gaussian"    # "gaussian" | "uniform" | "zipf"
+    act: str = "swiglu"          # "swiglu" (W13 [E, 2I, H]) | "relu2" (W1 [E, I, H])
 
     def with_T(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -58,10 +62,15 @@ class Workload:
     def R(self) -> int:
         return self.T * self.k
 
+    @property
+    def gemm1_rows(self) -> int:
+        """Weight rows per expert of GEMM1: 2I (gate + up) or I (ReLU2)."""
+        return self.I if self.act == "relu2" else 2 * self.I
+
     def flops(self) -> float:
-        """Routed-expert FLOPs of one forward pass: 2*H*2I (GEMM1) + 2*I*H (GEMM2) per
-        routed row (router, SwiGLU elementwise and combine excluded)."""
-        return 6.0 * self.T * self.k * self.H * self.I
+        """Routed-expert FLOPs of one forward pass: 2*H*(2I or I) (GEMM1) + 2*I*H (GEMM2)
+        per routed row (router, activation elementwise and combine excluded)."""
+        return 2.0 * self.T * self.k * self.H * (self.gemm1_rows + self.I)
 
 
 WORKLOADS = {
@@ -72,6 +81,7 @@ WORKLOADS = {
     "fp8_mxfp4": Workload("fp8_mxfp4", 8192, 2560, 640, 512, 10, dtype="fp8_mxfp4",
                           routing="uniform"),
     "decode": Workload("decode", 32, 4096, 14336, 8, 2, routing="zipf"),
+    "nemotron_relu2": Workload("nemotron_relu2", 8192, 2688, 1856, 128, 6, act="relu2"),
 }
 GRID = {f"grid_d{d}_e{e}_k{k}": Workload(f"grid_d{d}_e{e}_k{k}", 8192, d, d, e, k)
         for d in (2048, 4096) for e in (8, 16, 32, 64, 128) for k in (1, 2, 4, 8) if k < e}
@@ -92,14 +102,14 @@ def make_x(wl: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
 
 
 def make_weights(wl: Workload, seed: int = 0, device="cpu"):
-    """W13 bf16 [E, 2I, H] (gate rows then up rows) and W2 bf16 [E, H, I], drawn one
-    expert at a time to bound the temporary fp32 memory."""
+    """W13 bf16 [E, 2I, H] (gate rows then up rows; W1 [E, I, H] for ReLU2) and W2 bf16
+    [E, H, I], drawn one expert at a time to bound the temporary fp32 memory."""
     g = _gen(seed + 1, device)
-    w13 = torch.empty(wl.E, 2 * wl.I, wl.H, dtype=torch.bfloat16, device=device)
+    w13 = torch.empty(wl.E, wl.gemm1_rows, wl.H, dtype=torch.bfloat16, device=device)
     w2 = torch.empty(wl.E, wl.H, wl.I, dtype=torch.bfloat16, device=device)
     s13, s2 = 1.0 / math.sqrt(wl.H), 1.0 / math.sqrt(wl.I)
     for e in range(wl.E):
-        w13[e] = (torch.randn(2 * wl.I, wl.H, generator=g, device=device) * s13).to(torch.bfloat16)
+        w13[e] = (torch.randn(wl.gemm1_rows, wl.H, generator=g, device=device) * s13).to(torch.bfloat16)
     for e in range(wl.E):
         w2[e] = (torch.randn(wl.H, wl.I, generator=g, device=device) * s2).to(torch.bfloat16)
     return w13, w2

@@ -26,6 +26,11 @@ SMALL = {
     "sigmoid_top1": I.Workload("sig", 200, 512, 256, 16, 1, score="sigmoid", renorm=False),
     "zipf_empty_experts": I.Workload("zipf", 96, 512, 384, 8, 2, routing="zipf"),
     "many_tiles": I.Workload("many", 1000, 512, 256, 8, 4),
+    # ReLU2 (non-gated, W1 [E, I, H]): one partial 256-column tile (I = 192), two and a
+    # half tiles (I = 640), and a decode-sized batch (GEMM2 on the decode kernels)
+    "relu2_i192": I.Workload("r2a", 300, 256, 192, 8, 2, act="relu2"),
+    "relu2_i640": I.Workload("r2b", 1000, 512, 640, 8, 4, act="relu2"),
+    "relu2_t48": I.Workload("r2c", 48, 512, 256, 8, 2, act="relu2"),
 }
 
 
@@ -124,7 +129,7 @@ def test_gemm1_swiglu_parity(name):
     assert canary_intact(buf, R, wl.I)
     tok = or2a.astype(np.int64) // wl.k
     ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
-    ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), tok, ex)
+    ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), tok, ex, act=wl.act)
     assert_close(f64(act), ref, what=f"gemm1 {name}")
 
 
@@ -185,7 +190,7 @@ def _check_forward(wl, inp, logits, tokens, skew=False):
     oids, ow = oracle_route(wl, logits)
     assert np.array_equal(ids.cpu().numpy(), oids)
     ref, _ = oracle.forward_bf16(I.bits(inp["x"]), oids, ow, I.bits(inp["w13"]),
-                                 I.bits(inp["w2"]), tokens)
+                                 I.bits(inp["w2"]), tokens, act=wl.act)
     got = f64(out)[tokens]
     return assert_close(got, ref, COS_BF16, what=f"forward {wl.name} T={wl.T}"), (out, ws)
 
@@ -233,6 +238,7 @@ FULL = {
     # points of the parameter grid: 8192 rows per expert (top-1), 512 (E=128, top-8) and
     # 2048 at H=I=4096 -- single-SM and SM-pair GEMM2, K up to 4096
     **{n: W[n] for n in ("grid_d2048_e8_k1", "grid_d2048_e128_k8", "grid_d4096_e16_k4")},
+    "nemotron_relu2": W["nemotron_relu2"],
 }
 
 

@@ -58,6 +58,9 @@ def lib():
             L.orc_ue8m0_decode.argtypes = [u8]; L.orc_ue8m0_decode.restype = f64
             L.orc_route.argtypes = [i64, i32, i32, i32, i32, _P(f32), _P(ctypes.c_int32), _P(f64)]
             L.orc_route.restype = i32
+            L.orc_route_shared.argtypes = [i64, i32, i32, i32, i32, i32, _P(f32),
+                                           _P(ctypes.c_int32), _P(f64)]
+            L.orc_route_shared.restype = i32
             L.orc_permute.argtypes = [i64, i32, i32] + [_P(ctypes.c_int32)] * 5
             L.orc_permute.restype = i32
             L.orc_quant_fp8_rows.argtypes = [i64, i32, _P(f64), _P(u8), _P(f32)]
@@ -153,14 +156,21 @@ def ue8m0_decode(b) -> np.ndarray:
 SOFTMAX, SIGMOID = 0, 1
 
 
-def route(logits: np.ndarray, k: int, score: int = SOFTMAX, renorm: bool = True):
-    """Top-k by descending logit (ties to the lower index) and the slot weights (fp64)."""
+def route(logits: np.ndarray, k: int, score: int = SOFTMAX, renorm: bool = True,
+          n_shared: int = 0):
+    """Top-k by descending logit (ties to the lower index) and the slot weights (fp64);
+    with n_shared > 0, slots k.. hold the shared experts E.. with weight 1."""
     lg = _c(logits, np.float32)
     T, E = lg.shape
-    ids = np.empty((T, k), np.int32)
-    w = np.empty((T, k), np.float64)
-    rc = lib().orc_route(T, E, k, score, int(bool(renorm)), _ptr(lg, np.float32),
-                         _ptr(ids, np.int32), _ptr(w, np.float64))
+    ids = np.empty((T, k + n_shared), np.int32)
+    w = np.empty((T, k + n_shared), np.float64)
+    if n_shared:
+        rc = lib().orc_route_shared(T, E, k, n_shared, score, int(bool(renorm)),
+                                    _ptr(lg, np.float32), _ptr(ids, np.int32),
+                                    _ptr(w, np.float64))
+    else:
+        rc = lib().orc_route(T, E, k, score, int(bool(renorm)), _ptr(lg, np.float32),
+                             _ptr(ids, np.int32), _ptr(w, np.float64))
     if rc != 0:
         raise ValueError("orc_route: bad arguments")
     return ids, w

@@ -26,6 +26,9 @@
  *                -- read as the non-gated squared ReLU, the pages name only "ReLU2".
  *   combine      out[t] = sum over slots j (ascending) of w[t,j] * y_j, rounded once to
  *                bf16 (TileScale PR #70, the top-k slot reduction of kernel 2).
+ *   shared       n_shared always-on experts (index E + s) as extra slots of weight 1 after
+ *                the k routed ones (the pages fold shared experts into the compute; the
+ *                slot reading is this file's).
  *   block-scaled activations: FP8 e4m3 with one power-of-two fp32 scale per 1x128 group
  *                (TileScale PR #70, "Design": FP8 E4M3 with fp32 per-128-element
  *                scales); weights: MXFP4 e2m1 with one UE8M0 scale per 32 consecutive
@@ -168,6 +171,35 @@ int orc_route(int64_t T, int E, int k, int score, int renorm, const float *logit
   }
   free(sel);
   return 0;
+}
+
+/* Shared experts folded into the routed computation (GC-MoE "shared experts folded into
+ * the compute role"; DeepGEMM's "fused shared-expert execution" as the TileScale PR
+ * mentions it): experts E .. E+n_shared-1 run on every token with weight 1, read as
+ * extra slots k .. k+n_shared-1 appended after the k routed ones.  ids/w are
+ * [T][k + n_shared]. */
+int orc_route_shared(int64_t T, int E, int k, int n_shared, int score, int renorm,
+                     const float *logits, int32_t *ids, double *w) {
+  if (n_shared < 0) return -1;
+  const int ks = k + n_shared;
+  int32_t *rid = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * k + 1));
+  double *rw = (double *)malloc(sizeof(double) * (size_t)(T * k + 1));
+  if (!rid || !rw) { free(rid); free(rw); return -1; }
+  int rc = orc_route(T, E, k, score, renorm, logits, rid, rw);
+  if (rc == 0) {
+    for (int64_t t = 0; t < T; ++t) {
+      for (int j = 0; j < k; ++j) {
+        ids[t * ks + j] = rid[t * k + j];
+        w[t * ks + j] = rw[t * k + j];
+      }
+      for (int s = 0; s < n_shared; ++s) {
+        ids[t * ks + k + s] = E + s;
+        w[t * ks + k + s] = 1.0;
+      }
+    }
+  }
+  free(rid); free(rw);
+  return rc;
 }
 
 /* ------------------------------------------------------------------------------------ */

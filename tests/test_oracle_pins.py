@@ -398,6 +398,30 @@ def test_forward_relu2_brute_force_tiny(orc, T, E, k):
     assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
 
 
+def test_shared_experts_add_a_dense_mlp_to_the_routed_output(orc):
+    """Shared experts: the routed forward plus, for every token, each shared expert's
+    dense SwiGLU MLP with weight 1 (an independent numpy formulation)."""
+    rng = np.random.default_rng(23)
+    T, H, I, E, k, ns = 7, 64, 32, 5, 2, 2
+    xb = _rand_bf16(rng, (T, H))
+    w13 = _rand_bf16(rng, (E + ns, 2 * I, H), H ** -0.5)
+    w2 = _rand_bf16(rng, (E + ns, H, I), I ** -0.5)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    ids, w = orc.route(lg, k, n_shared=ns)
+    assert ids.shape == (T, k + ns)
+    assert np.array_equal(ids[:, k:], np.tile(np.arange(E, E + ns), (T, 1)))
+    assert np.array_equal(w[:, k:], np.ones((T, ns)))
+    rid, rw = orc.route(lg, k)
+    assert np.array_equal(ids[:, :k], rid) and np.array_equal(w[:, :k], rw)
+    out, _ = orc.forward_bf16(xb, ids, w, w13, w2)
+    xv, g13, g2 = _bits_to_f64(xb), _bits_to_f64(w13), _bits_to_f64(w2)
+    ref = _dense_moe_np(xv, lg, k, g13[:E], g2[:E])
+    for s_ in range(ns):
+        e = E + s_
+        ref += (_silu(xv @ g13[e, :I].T) * (xv @ g13[e, I:].T)) @ g2[e].T
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
+
+
 def test_forward_token_subset_and_order_equivariance(orc):
     rng = np.random.default_rng(21)
     T, H, I, E, k = 12, 32, 32, 5, 2

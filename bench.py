@@ -217,7 +217,7 @@ def stages_of(wl):
 
 def algorithmic(wl, counts):
     """Algorithmic FLOPs and bytes of each stage for the actual per-expert counts."""
-    T, H, Ii, E, k, R = wl.T, wl.H, wl.I, wl.E, wl.k, wl.R
+    T, H, Ii, E, k, R = wl.T, wl.H, wl.I, wl.E_all, wl.k + wl.n_shared, wl.R
     ne = int((counts > 0).sum())
     fp8 = wl.dtype == "fp8_mxfp4"
     wbytes = (0.5 + 1.0 / 32) if fp8 else 2.0     # per weight element (codes + scales)
@@ -253,10 +253,10 @@ def bench_ours(args, rank, world, local):
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device="cuda")
     R = wl.R
     bufs = {
-        "ids": torch.empty(wl.T, wl.k, dtype=torch.int32, device="cuda"),
-        "w": torch.empty(wl.T, wl.k, dtype=torch.float32, device="cuda"),
-        "counts": torch.empty(wl.E, dtype=torch.int32, device="cuda"),
-        "offsets": torch.empty(wl.E + 1, dtype=torch.int32, device="cuda"),
+        "ids": torch.empty(wl.T, wl.k + wl.n_shared, dtype=torch.int32, device="cuda"),
+        "w": torch.empty(wl.T, wl.k + wl.n_shared, dtype=torch.float32, device="cuda"),
+        "counts": torch.empty(wl.E_all, dtype=torch.int32, device="cuda"),
+        "offsets": torch.empty(wl.E_all + 1, dtype=torch.int32, device="cuda"),
         "r2a": torch.empty(R, dtype=torch.int32, device="cuda"),
         "a2r": torch.empty(R, dtype=torch.int32, device="cuda"),
         "act": torch.empty(R, wl.I, dtype=torch.bfloat16, device="cuda"),
@@ -407,10 +407,13 @@ def bench_ours(args, rank, world, local):
         "dtype": "e4m3 x e2m1 (fp32 accumulate)" if fp8 else "bf16",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, random-init)",
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                   **({"activation": wl.act} if wl.act != "swiglu" else {}),
+                   **({"n_shared": wl.n_shared} if wl.n_shared else {}),
                    "score": wl.score, "routing": wl.routing, "parallelism": f"replicas x{world}",
                    "nonempty_experts": ne,
                    "l2": "inputs larger than L2 (weights %.2f GB re-read every step)" %
-                         ((3 * wl.E * wl.I * wl.H * ((0.5 + 1 / 32) if fp8 else 2)) / 1e9)},
+                         (((wl.gemm1_rows + wl.I) * wl.E_all * wl.H * ((0.5 + 1 / 32) if fp8 else 2))
+                          / 1e9)},
         "hbm_gbs_alg": round(b_alg / (ms_max * 1e-3) / 1e9, 1),
         "hbm_frac_alg": round(b_alg / (ms_max * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "roofline": roof,
@@ -454,8 +457,8 @@ def cpu_baseline(wl, inp, budget_s=20.0, T_sample=None):
     wts = _oracle_weights(wl, inp)
     score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
     t0 = time.perf_counter()
-    ids, w = oracle.route(lg, wl.k, score, wl.renorm)
-    oracle.permute(ids, wl.E)
+    ids, w = oracle.route(lg, wl.k, score, wl.renorm, n_shared=wl.n_shared)
+    oracle.permute(ids, wl.E_all)
     t_route = time.perf_counter() - t0
     # probe the per-token cost on a few tokens, then size the sample for the budget
     probe = I.parity_tokens(wl.T, 4, seed=1)
@@ -491,7 +494,7 @@ def bench_reference(args, rank, world):
     lg = inp["logits"].cpu().numpy()
     wts = _oracle_weights(wl, inp)
     score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
-    ids, w = oracle.route(lg, wl.k, score, wl.renorm)
+    ids, w = oracle.route(lg, wl.k, score, wl.renorm, n_shared=wl.n_shared)
     probe = I.parity_tokens(wl.T, 4, seed=1)
     t0 = time.perf_counter()
     _oracle_forward(wl, x, ids, w, wts, probe)
@@ -502,13 +505,13 @@ def bench_reference(args, rank, world):
     for s in range(args.warmup + args.steps):
         toks = I.parity_tokens(wl.T, n, seed=10 + s)
         t0 = time.perf_counter()
-        oracle.route(lg, wl.k, score, wl.renorm)
+        oracle.route(lg, wl.k, score, wl.renorm, n_shared=wl.n_shared)
         _oracle_forward(wl, x, ids, w, wts, toks)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)
     sec = float(np.mean(times))
-    flops = 2.0 * n * wl.k * wl.H * (wl.gemm1_rows + wl.I)
+    flops = 2.0 * n * (wl.k + wl.n_shared) * wl.H * (wl.gemm1_rows + wl.I)
     val = flops / sec / 1e12
     return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -77,7 +77,14 @@ typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_MXFP4 = 1 } moe_dtype_t;
 typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act_t;
 
 /* Problem description.  score: moe_score_t; renormalize: 1 = divide the k selected
- * weights by their sum; dtype: moe_dtype_t; activation: moe_act_t. */
+ * weights by their sum; dtype: moe_dtype_t; activation: moe_act_t.
+ * n_shared: shared experts (0 = none), run on every token with weight 1 (GC-MoE folds
+ * shared experts into the compute role; DeepGEMM's SM100 path fuses them).  They are
+ * experts E .. E+n_shared-1 of the weight tensors (which then hold E + n_shared experts;
+ * logits stay [T][E]) and each token gets them as slots k .. k+n_shared-1 after its k
+ * routed ones: every "k" and "E" below, past routing's own top-k selection, means
+ * k + n_shared and E + n_shared (ids and w are [T][k + n_shared], R = T*(k + n_shared),
+ * counts [E + n_shared]).  k + n_shared <= 32 and E + n_shared <= 1024. */
 typedef struct {
   int64_t T;
   int32_t H, I, E, k;
@@ -85,6 +92,7 @@ typedef struct {
   int32_t renormalize;
   int32_t dtype;
   int32_t activation;
+  int32_t n_shared;
 } moe_shape_t;
 
 /* Bytes of device workspace moe_forward needs for `shape` (the stage entry points need

@@ -43,19 +43,20 @@ class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("activation", ctypes.c_int32)]
+                ("activation", ctypes.c_int32), ("n_shared", ctypes.c_int32)]
 
     @classmethod
     def of(cls, T, H, I, E, k, score="softmax", renorm=True, dtype="bf16",
-           act="swiglu") -> "MoeShape":
+           act="swiglu", n_shared=0) -> "MoeShape":
         return cls(int(T), int(H), int(I), int(E), int(k),
                    MOE_SCORE_SOFTMAX if score == "softmax" else MOE_SCORE_SIGMOID,
                    int(bool(renorm)), MOE_DTYPE_BF16 if dtype == "bf16" else MOE_DTYPE_FP8_MXFP4,
-                   MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_RELU2)
+                   MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_RELU2, int(n_shared))
 
     @classmethod
     def from_workload(cls, wl) -> "MoeShape":
-        return cls.of(wl.T, wl.H, wl.I, wl.E, wl.k, wl.score, wl.renorm, wl.dtype, wl.act)
+        return cls.of(wl.T, wl.H, wl.I, wl.E, wl.k, wl.score, wl.renorm, wl.dtype, wl.act,
+                      wl.n_shared)
 
 
 class MoeError(RuntimeError):

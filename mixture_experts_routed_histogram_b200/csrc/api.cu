@@ -22,6 +22,11 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
+// Shared experts are folded in as experts E .. E+n_shared-1 and slots k .. k+n_shared-1:
+// every stage after routing works on e_all experts and k_all slots per token.
+int e_all(const moe_shape_t& s) { return s.E + s.n_shared; }
+int k_all(const moe_shape_t& s) { return s.k + s.n_shared; }
+
 // Workspace regions (byte offsets from the workspace base).
 struct WsLayout {
   size_t status, ids, w, counts, offsets, r2a, a2r, scratch, xq, sx, sxw, act, act_sf, act_sfw,
@@ -29,7 +34,7 @@ struct WsLayout {
 };
 
 WsLayout layout(const moe_shape_t& s) {
-  const size_t T = static_cast<size_t>(s.T), R = T * s.k, H = s.H, I = s.I, E = s.E;
+  const size_t T = static_cast<size_t>(s.T), R = T * k_all(s), H = s.H, I = s.I, E = e_all(s);
   const bool fp8 = s.dtype == MOE_DTYPE_FP8_MXFP4;
   WsLayout L{};
   size_t o = 0;
@@ -40,7 +45,7 @@ WsLayout layout(const moe_shape_t& s) {
   L.offsets = o; o = up(o + 4 * (E + 1));
   L.r2a = o; o = up(o + 4 * R);
   L.a2r = o; o = up(o + 4 * R);
-  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(T), s.E));
+  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(T), e_all(s)));
   L.xq = o; o = up(o + (fp8 ? T * H : 0));
   L.sx = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
   L.sxw = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
@@ -66,9 +71,9 @@ moe_status_t check_shape(const moe_shape_t* s) {
     return MOE_ERR_INVALID_ARG;
   if (s->activation == MOE_ACT_RELU2 && s->dtype != MOE_DTYPE_BF16)
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
-  if (s->k > moe::kMaxTopK || s->E > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (s->T * static_cast<int64_t>(s->k) >= (static_cast<int64_t>(1) << 31))
+  if (s->k > s->E || s->n_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (k_all(*s) > moe::kMaxTopK || e_all(*s) > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->T * static_cast<int64_t>(k_all(*s)) >= (static_cast<int64_t>(1) << 31))
     return MOE_ERR_UNSUPPORTED_SHAPE;
   const int q = s->dtype == MOE_DTYPE_BF16 ? 64 : 128;
   if (s->H % q != 0 || s->I % q != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -94,11 +99,11 @@ moe_status_t need_ptrs(std::initializer_list<const void*> ps) {
 moe::GemmProblem problem(const moe_shape_t& s) {
   moe::GemmProblem p{};
   p.T = s.T;
-  p.R = s.T * s.k;
+  p.R = s.T * k_all(s);
   p.H = s.H;
   p.I = s.I;
-  p.E = s.E;
-  p.k = s.k;
+  p.E = e_all(s);
+  p.k = k_all(s);
   p.act = s.activation;
   p.wait_limit_ns = g_wait_limit_ns;
   return p;
@@ -136,7 +141,8 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* i
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({logits, ids, w}));
   int n = 0;
-  cudaError_t e = moe::launch_route(logits, ids, w, shape->T, shape->E, shape->k, shape->score,
+  cudaError_t e = moe::launch_route(logits, ids, w, shape->T, shape->E, shape->k,
+                                    shape->n_shared, shape->score,
                                     shape->renormalize, stream, &n);
   g_last_launches = n;
   return cuda_status(e);
@@ -148,13 +154,13 @@ moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* ids, int32_t* 
   g_last_launches = 0;
   MOE_TRY(check_shape(shape));
   MOE_TRY(need_ptrs({counts, offsets, ws}));
-  const int64_t R = shape->T * shape->k;
+  const int64_t R = shape->T * k_all(*shape);
   if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
   const WsLayout L = layout(*shape);
-  if (ws_bytes < L.scratch + moe::permute_scratch_bytes(shape->T, shape->E))
+  if (ws_bytes < L.scratch + moe::permute_scratch_bytes(shape->T, e_all(*shape)))
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   int n = 0;
-  cudaError_t e = moe::launch_permute(ids, shape->T, shape->k, shape->E, counts, offsets,
+  cudaError_t e = moe::launch_permute(ids, shape->T, k_all(*shape), e_all(*shape), counts, offsets,
                                       row2assign, assign2row, at<int32_t>(ws, L.scratch),
                                       status_word(ws), stream, &n);
   g_last_launches = n;
@@ -167,11 +173,11 @@ moe_status_t moe_permute_noalloc(const moe_shape_t* shape, const int32_t* ids, i
   g_last_launches = 0;
   MOE_TRY(check_shape(shape));
   MOE_TRY(need_ptrs({counts, offsets}));
-  const int64_t R = shape->T * shape->k;
+  const int64_t R = shape->T * k_all(*shape);
   if (R > 0) MOE_TRY(need_ptrs({ids, row2assign, assign2row}));
-  if (!moe::permute_noalloc_fits(shape->T, shape->E)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!moe::permute_noalloc_fits(shape->T, e_all(*shape))) return MOE_ERR_UNSUPPORTED_SHAPE;
   int n = 0;
-  cudaError_t e = moe::launch_permute_noalloc(ids, shape->T, shape->k, shape->E, counts, offsets,
+  cudaError_t e = moe::launch_permute_noalloc(ids, shape->T, k_all(*shape), e_all(*shape), counts, offsets,
                                               row2assign, assign2row, stream, &n);
   g_last_launches = n;
   return cuda_status(e);
@@ -254,7 +260,7 @@ moe_status_t moe_grouped_gemm2(const moe_shape_t* shape, const void* act, const 
     const WsLayout L = layout(*shape);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     uint32_t* asw = at<uint32_t>(ws, L.act_sfw);
-    const int64_t R = shape->T * shape->k;
+    const int64_t R = shape->T * k_all(*shape);
     cudaError_t e = moe::launch_scale_words(act_sf, asw, R * (shape->I / 128), stream, &n);
     if (e == cudaSuccess)
       e = moe::launch_gemm2_mx(problem(*shape), static_cast<const uint8_t*>(act), asw, offsets,
@@ -277,7 +283,7 @@ moe_status_t moe_combine(const moe_shape_t* shape, const uint16_t* y, const floa
   if (shape->T == 0) return MOE_OK;
   MOE_TRY(need_ptrs({y, w, assign2row, out}));
   int n = 0;
-  cudaError_t e = moe::launch_combine(y, w, assign2row, out, shape->T, shape->H, shape->k, stream,
+  cudaError_t e = moe::launch_combine(y, w, assign2row, out, shape->T, shape->H, k_all(*shape), stream,
                                       &n);
   g_last_launches = n;
   return cuda_status(e);
@@ -302,7 +308,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     if (!aligned32(w13) || !aligned32(w2)) return MOE_ERR_MISALIGNED;
   }
 
-  const int64_t T = shape->T, R = T * shape->k;
+  const int64_t T = shape->T, R = T * k_all(*shape);
   int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
   float* w = at<float>(ws, L.w);
   int32_t* counts = at<int32_t>(ws, L.counts);
@@ -315,16 +321,18 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
   const moe::GemmProblem p = problem(*shape);
   int n = 0;
   cudaError_t e;
-  if (moe::use_route_permute_small(T, shape->E, shape->k)) {
-    if ((e = moe::launch_route_permute_small(logits, T, shape->E, shape->k, shape->score,
+  if (moe::use_route_permute_small(T, e_all(*shape), k_all(*shape))) {
+    if ((e = moe::launch_route_permute_small(logits, T, shape->E, shape->k, shape->n_shared,
+                                             shape->score,
                                              shape->renormalize, ids, w, counts, offsets, r2a,
                                              a2r, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
   } else {
-    if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->score,
+    if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->n_shared,
+                               shape->score,
                                shape->renormalize, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if ((e = moe::launch_permute(ids, T, shape->k, shape->E, counts, offsets, r2a, a2r,
+    if ((e = moe::launch_permute(ids, T, k_all(*shape), e_all(*shape), counts, offsets, r2a, a2r,
                                  at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
@@ -358,7 +366,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
                                     splits, status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (splits > 1) {
-      if ((e = moe::launch_combine_parts(part, splits, R, w, a2r, out, T, shape->H, shape->k,
+      if ((e = moe::launch_combine_parts(part, splits, R, w, a2r, out, T, shape->H, k_all(*shape),
                                          stream, &n)) != cudaSuccess)
         return MOE_ERR_CUDA;
       g_last_launches = n;
@@ -372,7 +380,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
                                     stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
-  if ((e = moe::launch_combine(y, w, a2r, out, T, shape->H, shape->k, stream, &n)) !=
+  if ((e = moe::launch_combine(y, w, a2r, out, T, shape->H, k_all(*shape), stream, &n)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   g_last_launches = n;

@@ -12,9 +12,10 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 
-// Routing: ids/w [T][k] from logits [T][E].
+// Routing: ids/w [T][k + ns] from logits [T][E]: the top-k, then the ns shared experts
+// E .. E+ns-1 with weight 1.
 cudaError_t launch_route(const float* logits, int32_t* ids, float* w, int64_t T, int E, int k,
-                         int score, int renorm, cudaStream_t stream, int* launches);
+                         int ns, int score, int renorm, cudaStream_t stream, int* launches);
 
 // Histogram / prefix sum / stable scatter of the T*k assignments (chunks of 64 tokens,
 // fewer and larger chunks beyond 128 of them).  `scratch` holds the per-chunk histograms
@@ -34,10 +35,11 @@ cudaError_t launch_permute_noalloc(const int32_t* ids, int64_t T, int k, int E, 
 // Routing + histogram + prefix sum + stable scatter in one single-CTA launch, for
 // decode-sized batches (use_route_permute_small).  Same outputs as launch_route followed
 // by launch_permute.
-bool use_route_permute_small(int64_t T, int E, int k);
-cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int score,
-                                       int renorm, int32_t* ids, float* w, int32_t* counts,
-                                       int32_t* offsets, int32_t* row2assign,
+// (E, k: routed experts and top-k; ns shared experts are appended as in launch_route.)
+bool use_route_permute_small(int64_t T, int E_all, int k_all);
+cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int ns,
+                                       int score, int renorm, int32_t* ids, float* w,
+                                       int32_t* counts, int32_t* offsets, int32_t* row2assign,
                                        int32_t* assign2row, cudaStream_t stream, int* launches);
 
 // Weighted top-k combine.

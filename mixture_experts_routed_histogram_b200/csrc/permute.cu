@@ -265,8 +265,9 @@ namespace {
 
 template <int VPT>
 __global__ void __launch_bounds__(kSmallThreads)
-    route_permute_small_kernel(const float* __restrict__ logits, int T, int E, int k, int score,
-                               int renorm, int32_t* __restrict__ ids, float* __restrict__ w,
+    route_permute_small_kernel(const float* __restrict__ logits, int T, int E, int k, int ns,
+                               int score, int renorm, int32_t* __restrict__ ids,
+                               float* __restrict__ w,
                                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                int32_t* __restrict__ row2assign,
                                int32_t* __restrict__ assign2row) {
@@ -276,7 +277,9 @@ __global__ void __launch_bounds__(kSmallThreads)
   __shared__ int wcnt[kSmallWarps][kSmallMaxE];
   __shared__ int warp_sums[kSmallWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int R = T * k;
+  const int ks = k + ns;        // slots per token: the top-k, then the shared experts
+  const int Ea = E + ns;        // experts of the permutation
+  const int R = T * ks;
   pdl_wait();
   pdl_launch_dependents();
 
@@ -285,13 +288,17 @@ __global__ void __launch_bounds__(kSmallThreads)
     float wt;
     route_token_warp<VPT>(logits + static_cast<int64_t>(t) * E, E, k, score, renorm, lane, id,
                           wt);
-    if (lane < k) {
-      ids[t * k + lane] = id;
-      w[t * k + lane] = wt;
-      s_ids[t * k + lane] = id;
+    if (lane >= k) {
+      id = E + (lane - k);
+      wt = 1.0f;
+    }
+    if (lane < ks) {
+      ids[t * ks + lane] = id;
+      w[t * ks + lane] = wt;
+      s_ids[t * ks + lane] = id;
     }
   }
-  for (int e = tid; e < E; e += kSmallThreads) {
+  for (int e = tid; e < Ea; e += kSmallThreads) {
     scan[e] = 0;
 #pragma unroll 4
     for (int ww = 0; ww < kSmallWarps; ++ww) wcnt[ww][e] = -1;
@@ -299,8 +306,8 @@ __global__ void __launch_bounds__(kSmallThreads)
   __syncthreads();
   for (int a = tid; a < R; a += kSmallThreads) atomicAdd(&scan[s_ids[a]], 1);
   __syncthreads();
-  // exclusive scan of the E counts: one per thread, warp scans, then the warp totals
-  const int cnt = tid < E ? scan[tid] : 0;
+  // exclusive scan of the Ea counts: one per thread, warp scans, then the warp totals
+  const int cnt = tid < Ea ? scan[tid] : 0;
   int incl = cnt;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -312,12 +319,12 @@ __global__ void __launch_bounds__(kSmallThreads)
   int before = 0;
   for (int ww = 0; ww < warp; ++ww) before += warp_sums[ww];
   const int excl = before + incl - cnt;
-  if (tid < E) {
+  if (tid < Ea) {
     cursor[tid] = excl;
     offsets[tid] = excl;
     counts[tid] = cnt;
   }
-  if (tid == 0) offsets[E] = R;
+  if (tid == 0) offsets[Ea] = R;
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
   for (int r = 0; r * kSmallThreads < R; ++r) {
@@ -345,37 +352,37 @@ __global__ void __launch_bounds__(kSmallThreads)
 }
 
 template <int VPT>
-cudaError_t launch_small(const float* logits, int T, int E, int k, int score, int renorm,
+cudaError_t launch_small(const float* logits, int T, int E, int k, int ns, int score, int renorm,
                          int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
                          int32_t* row2assign, int32_t* assign2row, cudaStream_t stream) {
   return launch_k(route_permute_small_kernel<VPT>, dim3(1), dim3(kSmallThreads), 0, stream, logits,
-                  T, E, k, score, renorm, ids, w, counts, offsets, row2assign, assign2row);
+                  T, E, k, ns, score, renorm, ids, w, counts, offsets, row2assign, assign2row);
 }
 
 }  // namespace
 
-bool use_route_permute_small(int64_t T, int E, int k) {
-  return T > 0 && T <= kSmallMaxT && E <= kSmallMaxE && k <= kMaxTopK;
+bool use_route_permute_small(int64_t T, int E_all, int k_all) {
+  return T > 0 && T <= kSmallMaxT && E_all <= kSmallMaxE && k_all <= kMaxTopK;
 }
 
-cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int score,
-                                       int renorm, int32_t* ids, float* w, int32_t* counts,
-                                       int32_t* offsets, int32_t* row2assign,
+cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, int k, int ns,
+                                       int score, int renorm, int32_t* ids, float* w,
+                                       int32_t* counts, int32_t* offsets, int32_t* row2assign,
                                        int32_t* assign2row, cudaStream_t stream, int* launches) {
   ++*launches;
   const int t = static_cast<int>(T);
   const int need = (E + 31) / 32;
   if (need <= 1)
-    return launch_small<1>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
-                           assign2row, stream);
+    return launch_small<1>(logits, t, E, k, ns, score, renorm, ids, w, counts, offsets,
+                           row2assign, assign2row, stream);
   if (need <= 2)
-    return launch_small<2>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
-                           assign2row, stream);
+    return launch_small<2>(logits, t, E, k, ns, score, renorm, ids, w, counts, offsets,
+                           row2assign, assign2row, stream);
   if (need <= 4)
-    return launch_small<4>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
-                           assign2row, stream);
-  return launch_small<8>(logits, t, E, k, score, renorm, ids, w, counts, offsets, row2assign,
-                         assign2row, stream);
+    return launch_small<4>(logits, t, E, k, ns, score, renorm, ids, w, counts, offsets,
+                           row2assign, assign2row, stream);
+  return launch_small<8>(logits, t, E, k, ns, score, renorm, ids, w, counts, offsets,
+                         row2assign, assign2row, stream);
 }
 
 // ---------------------------------------------------------------- allocation-free variant

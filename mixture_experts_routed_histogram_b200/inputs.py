@@ -17,6 +17,9 @@ Workloads (shapes and value recipes):
   nemotron_relu2  T=8192, H=2688, E=128, k=6, I=1856, ReLU2 (non-gated squared ReLU, W1
                   [E, I, H]), softmax top-6 renormalised, gaussian routing: the
                   Nemotron-3.5-Lightning shape FlashInfer PR #5129 measures.
+  qwen3_30b_a3b_shared1
+                  the Qwen3-30B-A3B shape plus one shared expert (expert 128, weight 1 on
+                  every token): the shared-expert fold at a realistic size.
   grid_d{D}_e{E}_k{k}
                   the parameter grid of the Liger-Kernel PR #1463 benchmark: T=8192,
                   H=I=D in {2048, 4096}, E in {8, 16, 32, 64, 128}, k in {1, 2, 4, 8} with
@@ -54,13 +57,19 @@ class Workload:
     dtype: str = "bf16"          # "bf16" | "fp8_mxfp4"
     routing: str = "gaussian"    # "gaussian" | "uniform" | "zipf"
     act: str = "swiglu"          # "swiglu" (W13 [E, 2I, H]) | "relu2" (W1 [E, I, H])
+    n_shared: int = 0            # shared experts E .. E+n_shared-1 (weights hold E + n_shared)
 
     def with_T(self, T: int) -> "Workload":
         return replace(self, T=T)
 
     @property
     def R(self) -> int:
-        return self.T * self.k
+        """Rows of the expert-sorted space: routed and shared slots of every token."""
+        return self.T * (self.k + self.n_shared)
+
+    @property
+    def E_all(self) -> int:
+        return self.E + self.n_shared
 
     @property
     def gemm1_rows(self) -> int:
@@ -68,9 +77,10 @@ class Workload:
         return self.I if self.act == "relu2" else 2 * self.I
 
     def flops(self) -> float:
-        """Routed-expert FLOPs of one forward pass: 2*H*(2I or I) (GEMM1) + 2*I*H (GEMM2)
-        per routed row (router, activation elementwise and combine excluded)."""
-        return 2.0 * self.T * self.k * self.H * (self.gemm1_rows + self.I)
+        """Expert FLOPs of one forward pass: 2*H*(2I or I) (GEMM1) + 2*I*H (GEMM2) per row
+        of the expert-sorted space (routed slots, plus the shared experts' when there are
+        any; router, activation elementwise and combine excluded)."""
+        return 2.0 * self.R * self.H * (self.gemm1_rows + self.I)
 
 
 WORKLOADS = {
@@ -82,6 +92,8 @@ WORKLOADS = {
                           routing="uniform"),
     "decode": Workload("decode", 32, 4096, 14336, 8, 2, routing="zipf"),
     "nemotron_relu2": Workload("nemotron_relu2", 8192, 2688, 1856, 128, 6, act="relu2"),
+    "qwen3_30b_a3b_shared1": Workload("qwen3_30b_a3b_shared1", 8192, 2048, 768, 128, 8,
+                                      n_shared=1),
 }
 GRID = {f"grid_d{d}_e{e}_k{k}": Workload(f"grid_d{d}_e{e}_k{k}", 8192, d, d, e, k)
         for d in (2048, 4096) for e in (8, 16, 32, 64, 128) for k in (1, 2, 4, 8) if k < e}
@@ -105,12 +117,12 @@ def make_weights(wl: Workload, seed: int = 0, device="cpu"):
     """W13 bf16 [E, 2I, H] (gate rows then up rows; W1 [E, I, H] for ReLU2) and W2 bf16
     [E, H, I], drawn one expert at a time to bound the temporary fp32 memory."""
     g = _gen(seed + 1, device)
-    w13 = torch.empty(wl.E, wl.gemm1_rows, wl.H, dtype=torch.bfloat16, device=device)
-    w2 = torch.empty(wl.E, wl.H, wl.I, dtype=torch.bfloat16, device=device)
+    w13 = torch.empty(wl.E_all, wl.gemm1_rows, wl.H, dtype=torch.bfloat16, device=device)
+    w2 = torch.empty(wl.E_all, wl.H, wl.I, dtype=torch.bfloat16, device=device)
     s13, s2 = 1.0 / math.sqrt(wl.H), 1.0 / math.sqrt(wl.I)
-    for e in range(wl.E):
+    for e in range(wl.E_all):
         w13[e] = (torch.randn(wl.gemm1_rows, wl.H, generator=g, device=device) * s13).to(torch.bfloat16)
-    for e in range(wl.E):
+    for e in range(wl.E_all):
         w2[e] = (torch.randn(wl.H, wl.I, generator=g, device=device) * s2).to(torch.bfloat16)
     return w13, w2
 
@@ -138,11 +150,11 @@ def make_weights_mxfp4(wl: Workload, seed: int = 0, device="cpu"):
     """MXFP4 W13 (packed [E, 2I, H/2] + scales [E, 2I, H/32]) and W2 (packed [E, H, I/2] +
     scales [E, H, I/32]), element 2i in the low nibble of byte i."""
     g = _gen(seed + 3, device)
-    w13p = torch.empty(wl.E, 2 * wl.I, wl.H // 2, dtype=torch.uint8, device=device)
-    w13s = torch.empty(wl.E, 2 * wl.I, wl.H // 32, dtype=torch.uint8, device=device)
-    w2p = torch.empty(wl.E, wl.H, wl.I // 2, dtype=torch.uint8, device=device)
-    w2s = torch.empty(wl.E, wl.H, wl.I // 32, dtype=torch.uint8, device=device)
-    for e in range(wl.E):
+    w13p = torch.empty(wl.E_all, 2 * wl.I, wl.H // 2, dtype=torch.uint8, device=device)
+    w13s = torch.empty(wl.E_all, 2 * wl.I, wl.H // 32, dtype=torch.uint8, device=device)
+    w2p = torch.empty(wl.E_all, wl.H, wl.I // 2, dtype=torch.uint8, device=device)
+    w2s = torch.empty(wl.E_all, wl.H, wl.I // 32, dtype=torch.uint8, device=device)
+    for e in range(wl.E_all):
         w13p[e], w13s[e] = _mx_block(2 * wl.I, wl.H, wl.H, g, device)
         w2p[e], w2s[e] = _mx_block(wl.H, wl.I, wl.I, g, device)
     return w13p, w13s, w2p, w2s

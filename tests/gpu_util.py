@@ -66,11 +66,11 @@ def routing_logits(wl: I.Workload, x: torch.Tensor, seed=0):
 
 def oracle_route(wl: I.Workload, logits: torch.Tensor):
     score = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
-    return oracle.route(logits.cpu().numpy(), wl.k, score, wl.renorm)
+    return oracle.route(logits.cpu().numpy(), wl.k, score, wl.renorm, n_shared=wl.n_shared)
 
 
 def gpu_route(shape, logits):
-    T, k = shape.T, shape.k
+    T, k = shape.T, shape.k + shape.n_shared
     ids = torch.empty(T, k, dtype=torch.int32, device=dev())
     w = torch.empty(T, k, dtype=torch.float32, device=dev())
     C.moe_route(shape, logits, ids, w)
@@ -78,7 +78,7 @@ def gpu_route(shape, logits):
 
 
 def gpu_permute(shape, ids, ws):
-    R, E = shape.T * shape.k, shape.E
+    R, E = shape.T * (shape.k + shape.n_shared), shape.E + shape.n_shared
     counts = torch.empty(E, dtype=torch.int32, device=dev())
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev())
     r2a = torch.empty(max(R, 1), dtype=torch.int32, device=dev())

@@ -30,7 +30,7 @@ CASES = {
 def _setup(wl):
     inp = I.make_inputs(wl, 0, dev())
     oids, _ = oracle_route(wl, inp["logits"])
-    _, oo, or2a, _ = oracle.permute(oids, wl.E)
+    _, oo, or2a, _ = oracle.permute(oids, wl.E_all)
     shape = C.MoeShape.from_workload(wl)
     ws = workspace(shape)
     fp8 = wl.dtype == "fp8_mxfp4"
@@ -93,7 +93,7 @@ def test_injected_stall_reports_timeout_and_context_survives(case, which):
     assert torch.equal(again.view(torch.uint8), clean.view(torch.uint8)), "results changed"
     if case == "bf16_swap":   # and the clean result is the oracle's
         inp, oo, or2a = st["inp"], st["oo"], st["or2a"]
-        ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+        ex = np.repeat(np.arange(wl.E_all), np.diff(oo)).astype(np.int32)
         if which == "gemm1":
             ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), or2a // wl.k, ex)
         else:

@@ -74,7 +74,7 @@ SMALL = {
 
 def _routing(wl, inp):
     oids, ow = oracle_route(wl, inp["logits"])
-    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E)
+    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E_all)
     return oids, ow, oo, or2a, oa2r
 
 
@@ -96,8 +96,8 @@ def test_gemm1_fp8_parity(name):
     torch.cuda.synchronize()
     assert C.moe_get_device_status(ws) == 0
     assert bool((act[R * wl.I:] == 0x5A).all())
-    tok = or2a.astype(np.int64) // wl.k
-    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    tok = or2a.astype(np.int64) // (wl.k + wl.n_shared)
+    ex = np.repeat(np.arange(wl.E_all), np.diff(oo)).astype(np.int32)
     exact = oracle.gemm1_fp8_rows(xq_np, sx_np, _np(inp["w13"]), _np(inp["w13_sf"]), tok, ex,
                                   requant_act=False)
     scales = np.repeat(_np(act_sf).astype(np.float64), 128, axis=1)
@@ -129,7 +129,7 @@ def test_gemm2_fp8_parity(name):
     torch.cuda.synchronize()
     assert C.moe_get_device_status(ws) == 0
     assert canary_intact(buf, R, wl.H)
-    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    ex = np.repeat(np.arange(wl.E_all), np.diff(oo)).astype(np.int32)
     ref = oracle.gemm2_fp8_rows(aq_np, sa_np, _np(inp["w2"]), _np(inp["w2_sf"]), np.arange(R), ex)
     assert_close(f64(y), ref, COS_BF16, what=f"gemm2 fp8 {name}")
 
@@ -141,7 +141,7 @@ def _forward_check(wl, tokens, weights_from_gpu_quantiser=False):
     shape = C.MoeShape.from_workload(wl)
     ws = workspace(shape)
     buf, out = with_canary(wl.T, wl.H)
-    ids = torch.empty(wl.T, wl.k, dtype=torch.int32, device=dev())
+    ids = torch.empty(wl.T, wl.k + wl.n_shared, dtype=torch.int32, device=dev())
     C.moe_forward(shape, inp["x"], inp["logits"], inp["w13"], inp["w13_sf"], inp["w2"],
                   inp["w2_sf"], out, ids, ws)
     torch.cuda.synchronize()

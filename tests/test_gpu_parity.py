@@ -31,6 +31,9 @@ SMALL = {
     "relu2_i192": I.Workload("r2a", 300, 256, 192, 8, 2, act="relu2"),
     "relu2_i640": I.Workload("r2b", 1000, 512, 640, 8, 4, act="relu2"),
     "relu2_t48": I.Workload("r2c", 48, 512, 256, 8, 2, act="relu2"),
+    # shared experts: experts E.. on every token with weight 1 (decode-sized and large)
+    "shared1_t40": I.Workload("sh1", 40, 256, 128, 8, 2, n_shared=1),
+    "shared2_t500": I.Workload("sh2", 500, 512, 256, 16, 4, n_shared=2),
 }
 
 
@@ -49,6 +52,8 @@ ROUTE_CASES = {
     "fp8_mxfp4_T16384": W["fp8_mxfp4"].with_T(16384),
     "decode_T256": W["decode"].with_T(256),
     "e1000_k32": I.Workload("wide", 300, 256, 128, 1000, 32),
+    "e16_k4_shared2": I.Workload("shr", 300, 256, 128, 16, 4, n_shared=2),
+    "e8_k2_shared1_t40": I.Workload("shs", 40, 256, 128, 8, 2, n_shared=1),
 }
 
 
@@ -67,7 +72,7 @@ def test_route_and_permute_bitexact(name):
     ws = workspace(shape)
     # permutation of the oracle's ids (an input independent of the CUDA path)
     counts, offsets, r2a, a2r = gpu_permute(shape, to_dev_i32(oids), ws)
-    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E)
+    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E_all)
     assert np.array_equal(counts.cpu().numpy(), oc)
     assert np.array_equal(offsets.cpu().numpy(), oo)
     assert np.array_equal(r2a.cpu().numpy(), or2a)
@@ -106,7 +111,7 @@ def _stage_inputs(wl, skew=False):
     inp = I.make_inputs(wl, 0, dev())
     lg = _skewed_logits(wl, inp["x"]) if skew else inp["logits"]
     oids, ow = oracle_route(wl, lg)
-    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E)
+    oc, oo, or2a, oa2r = oracle.permute(oids, wl.E_all)
     return inp, oids, ow, oo, or2a, oa2r
 
 
@@ -127,8 +132,8 @@ def test_gemm1_swiglu_parity(name):
     torch.cuda.synchronize()
     assert C.moe_get_device_status(ws) == 0
     assert canary_intact(buf, R, wl.I)
-    tok = or2a.astype(np.int64) // wl.k
-    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    tok = or2a.astype(np.int64) // (wl.k + wl.n_shared)
+    ex = np.repeat(np.arange(wl.E_all), np.diff(oo)).astype(np.int32)
     ref = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), tok, ex, act=wl.act)
     assert_close(f64(act), ref, what=f"gemm1 {name}")
 
@@ -147,7 +152,7 @@ def test_gemm2_parity(name):
     torch.cuda.synchronize()
     assert C.moe_get_device_status(ws) == 0
     assert canary_intact(buf, R, wl.H)
-    ex = np.repeat(np.arange(wl.E), np.diff(oo)).astype(np.int32)
+    ex = np.repeat(np.arange(wl.E_all), np.diff(oo)).astype(np.int32)
     ref = oracle.gemm2_bf16_rows(I.bits(act), I.bits(inp["w2"]), np.arange(R), ex)
     assert_close(f64(y), ref, what=f"gemm2 {name}")
 
@@ -175,7 +180,7 @@ def test_combine_parity(name):
 def _forward(wl, inp, logits, ws):
     shape = C.MoeShape.from_workload(wl)
     buf, out = with_canary(wl.T, wl.H)
-    ids = torch.empty(wl.T, wl.k, dtype=torch.int32, device=dev())
+    ids = torch.empty(wl.T, wl.k + wl.n_shared, dtype=torch.int32, device=dev())
     C.moe_forward(shape, inp["x"], logits, inp["w13"], None, inp["w2"], None, out, ids, ws)
     torch.cuda.synchronize()
     assert canary_intact(buf, wl.T, wl.H)
@@ -239,6 +244,7 @@ FULL = {
     # 2048 at H=I=4096 -- single-SM and SM-pair GEMM2, K up to 4096
     **{n: W[n] for n in ("grid_d2048_e8_k1", "grid_d2048_e128_k8", "grid_d4096_e16_k4")},
     "nemotron_relu2": W["nemotron_relu2"],
+    "qwen3_30b_a3b_shared1": W["qwen3_30b_a3b_shared1"],
 }
 
 

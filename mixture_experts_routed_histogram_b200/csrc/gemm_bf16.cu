@@ -1,6 +1,7 @@
 // gemm_bf16.cu -- grouped GEMMs over the expert-sorted row space on sm_100a tensor cores.
 //
 //   GEMM1 + SwiGLU: act[r][i] = silu(x[tok(r)] . W13[e][i]) * (x[tok(r)] . W13[e][I+i])
+//   GEMM1 + ReLU2:  act[r][i] = max(x[tok(r)] . W1[e][i], 0)^2
 //   GEMM2:          y[r][o]   = act[r] . W2[e][o]
 //
 // Sources: TileScale PR #70 (distributed FP8 MegaMoE), "Design" -- kernel 1 is GEMM1 with
@@ -10,17 +11,21 @@
 // BF16 fused MoE), "sorted I/O": GEMM1 gathers token rows for A and writes expert-sorted
 // rows, which GEMM2 reads as a contiguous A operand.
 //
-// B200 design (one persistent CTA per SM, 6 warps):
+// B200 design (one persistent CTA per SM; 6 warps, plus 4 loader warps for GEMM1):
 //   warp 0      producer: TMA loads into a STAGES-deep shared-memory ring guarded by
-//               full/empty mbarriers.  GEMM1's A tile is gathered with tile::gather4 (each
-//               lane fetches 4 token rows of 128 B); B is a 2-D tile load (GEMM1: the 128
-//               gate rows and the matching 128 up rows of one expert, stacked).
+//               full/empty mbarriers.  B is a 2-D tile load (GEMM1 SwiGLU: the 128 gate
+//               rows and the matching 128 up rows of one expert, stacked; ReLU2: 256
+//               consecutive W1 rows); GEMM2's A is a 2-D tile of the sorted act rows.
+//   warps 6-9   GEMM1 only: gather the tile's token rows of x with 16-byte cp.async into
+//               the 128-byte-swizzled layout (tile::gather4 by the producer instead is a
+//               tuning switch, MOE_GEMM1_GATHER=tma4, measured slower).
 //   warp 1      TMEM owner + MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16, bf16 -> fp32) into one of two TMEM accumulators, commits each stage
 //               back to its empty barrier and each finished tile to the epilogue.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp owns its 32-lane TMEM
-//               quadrant = 32 rows), SwiGLU (GEMM1) or plain conversion (GEMM2) to bf16,
-//               predicated row stores; then frees the accumulator for the next tile.
+//               quadrant = 32 rows), SwiGLU or ReLU2 (GEMM1) or plain conversion (GEMM2)
+//               to bf16, each 32x32 chunk staged in shared memory and stored by TMA
+//               (epilogue.cuh); then frees the accumulator for the next tile.
 // Tasks are a flat (expert, n-tile, m-tile) queue built in shared memory from the
 // expert offsets: CTA c takes tasks c, c + gridDim, ...  Consecutive tasks share the
 // same weight tile (n-tile) of one expert, so the SMs working at the same time read each

@@ -17,13 +17,16 @@
 //     per B row, which TMA unpacks to 128 bytes: 16 codes + an 8-byte gap per 16 bytes);
 //   * the activation scale of a stage is one 1x128 group, i.e. the same UE8M0 byte for all
 //     four K32 blocks; weight scales are K32 bytes as prepared;
-//   * scale factors of a stage are gathered with 4-byte cp.async into the 512-byte atom
-//     the MMA expects (row r at byte 16*(r%32) + 4*(r/32), one byte per K32 block), then
-//     copied into a per-stage TMEM slot with tcgen05.cp before the stage's four MMAs;
+//   * the scale factors of a stage sit in 512-byte atoms laid out as the MMA expects (row
+//     r at byte 16*(r%32) + 4*(r/32), one byte per K32 block) and are copied into a
+//     per-stage TMEM slot with tcgen05.cp before the stage's four MMAs.  GEMM1's loader
+//     threads read their rows' scale words four stages ahead with plain 16-byte loads and
+//     store them into the atoms; GEMM2's scale warp gathers them with 4-byte cp.async;
 //   * GEMM1 tiles are 128 rows x (128 gate + 128 up) columns so that the SwiGLU output of a
 //     tile is exactly one 1x128 requantisation group per row; its accumulator (256 TMEM
-//     columns) is single-buffered to leave room for the scale slots.  GEMM2 tiles are
-//     128 x 128 with a double-buffered accumulator.
+//     columns) is single-buffered to leave room for the scale slots, and the epilogue
+//     hands it back as soon as it has read it.  GEMM2 tiles are 128 x 256 the same way
+//     (H % 256 == 0), else 128 x 128 with a double-buffered accumulator.
 #include <cudaTypedefs.h>
 
 #include <mutex>

@@ -39,15 +39,16 @@ METRIC = "routed MoE MLP fwd TFLOP/s on 1 B200 at T=8192; µs/layer at decode T"
 PUBLISHED = {"qwen3_30b_a3b": 599.60}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernels, from the ncu captures summarised in profiles/ (gemm_bf16_qwen3_30b_a3b_T8192,
-# gemm_swap_decode_T1, gemm_mx_swap_fp8_mxfp4_T128, gemm_mx_fp8_mxfp4_T8192); an entry is
-# removed when its kernel changes after the capture.
+# kernels, from the ncu captures summarised in profiles/ (the DRAM-bytes pass of
+# dram_traffic_current_kernels, and gemm_mx_fp8_mxfp4_T8192); an entry is removed when its
+# kernel changes after the capture.
 NCU_TRAFFIC = {
-    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 968.51e6 + 94.64e6,
-    ("qwen3_30b_a3b", 8192, "gemm2"): 503.43e6 + 238.33e6,
-    ("decode", 1, "gemm1_swiglu"): 469.82e6 + 4.16e6,
-    ("decode", 1, "gemm2"): 234.98e6 + 3.68e6,
-    ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.71e6 + 4.96e6,
+    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 969.63e6 + 91.17e6,
+    ("qwen3_30b_a3b", 8192, "gemm2"): 503.41e6 + 234.69e6,
+    ("decode", 1, "gemm1_swiglu"): 469.82e6 + 0.44e6,
+    ("decode", 1, "gemm2"): 234.98e6 + 0.20e6,
+    ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.71e6 + 0.98e6,
+    ("fp8_mxfp4", 128, "gemm2"): 446.54e6 + 5.48e6,
     ("fp8_mxfp4", 8192, "gemm1_swiglu"): 1180.74e6 + 55.53e6,
     ("fp8_mxfp4", 8192, "gemm2"): 500.67e6 + 380.47e6,
 }

@@ -41,6 +41,9 @@ def _shape(moelib, **kw):
     (dict(k=0), 1), (dict(k=9), 1), (dict(T=-1), 1), (dict(H=0), 1),
     (dict(E=2000, k=2), 2), (dict(k=33, E=64), 2), (dict(H=100), 2), (dict(I=96), 2),
     (dict(dtype="fp8_mxfp4", H=192), 2), (dict(T=2 ** 29, k=8), 2),
+    # ReLU2 is BF16 only; shared experts count against the slot and expert limits
+    (dict(dtype="fp8_mxfp4", act="relu2"), 2), (dict(n_shared=-1), 1),
+    (dict(k=30, E=64, n_shared=3), 2), (dict(E=1023, n_shared=2), 2),
 ])
 def test_shape_validation(moelib, kw, status):
     L = moelib.load()
@@ -49,6 +52,21 @@ def test_shape_validation(moelib, kw, status):
     assert L.moe_route(ctypes.byref(s), 16, 16, 16, None) == status
     assert L.moe_forward(ctypes.byref(s), 16, 16, 16, None, 16, None, 16, None, 256, 1 << 30,
                          None) == status
+
+
+def test_unknown_activation_is_rejected(moelib):
+    L = moelib.load()
+    s = _shape(moelib)
+    s.activation = 7
+    assert L.moe_workspace_size(ctypes.byref(s)) == 0
+    assert L.moe_route(ctypes.byref(s), 16, 16, 16, None) == moelib.MOE_ERR_INVALID_ARG
+
+
+def test_shared_experts_grow_the_routed_row_space(moelib):
+    L = moelib.load()
+    a = L.moe_workspace_size(ctypes.byref(_shape(moelib, T=256)))
+    b = L.moe_workspace_size(ctypes.byref(_shape(moelib, T=256, n_shared=1)))
+    assert b - a >= 256 * (256 + 128) * 2          # one more row of act and y per token
 
 
 def test_pointer_validation(moelib):

@@ -388,6 +388,11 @@ def bench_ours(args, rank, world, local):
         roof = {"bound": "hbm", "achieved": bytes_s[dname] / t_ker / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    if roof["bound"] == "tensor":
+        # context: the same kernel against the power-capped, seconds-long cuBLAS figure
+        roof["frac_of_sustained"] = roof["achieved"] / (
+            pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) *
+            (2.0 if fp8 else 1.0))
     roof["traffic"] = NCU_TRAFFIC.get((wl.name, wl.T, dname))
     roof["traffic_unit"] = "bytes per launch (ncu)"
     roof["kernel"] = dname

@@ -506,8 +506,13 @@ bool tmap_mxs(CUtensorMap* m, const void* ptr, bool fp4, uint64_t inner, uint64_
 template <bool GEMM1, int NT, int NW2>
 cudaError_t run_mxs(const CUtensorMap& w, const CUtensorMap& t, const MxSwapArgs& a,
                     cudaStream_t stream) {
+  // as many stages as shared memory holds beside the reduction buffer and the bookkeeping
+  // (two barriers per stage, five more, the expert offsets and tile starts, 1 KB of
+  // alignment slack): the FP4 weight tiles take twice their HBM bytes once unpacked, so the
+  // ring depth is what keeps enough HBM data in flight per SM
   using C1 = MxSwapCfg<GEMM1, NT, 1, NW2>;
-  constexpr int STAGES0 = (190 * 1024 - C1::RED_BYTES) / (C1::STAGE + C1::SF_BYTES);
+  constexpr int FIXED = C1::RED_BYTES + 5 * 8 + 16 + 8 * (kMaxExperts + 1) + 1024;
+  constexpr int STAGES0 = (227 * 1024 - FIXED) / (C1::STAGE + C1::SF_BYTES + 16);
   constexpr int STAGES = STAGES0 > 8 ? 8 : STAGES0;
   using Cf = MxSwapCfg<GEMM1, NT, STAGES, NW2>;
   auto kern = mx_swap_gemm_kernel<GEMM1, NT, STAGES, NW2>;

@@ -473,9 +473,11 @@ bool tmap_bf16_swap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ou
 template <bool GEMM1, int NT>
 cudaError_t run_swap(const CUtensorMap& w, const CUtensorMap& t, const SwapArgs& args,
                      cudaStream_t stream) {
-  // fill shared memory with stages after the gate buffer and the bookkeeping (~9 KB)
-  constexpr int STAGES =
-      (190 * 1024 - SwapCfg<GEMM1, NT, 1>::GBUF_BYTES) / SwapCfg<GEMM1, NT, 1>::STAGE;
+  // fill shared memory with stages after the gate buffer and the bookkeeping (two barriers
+  // per stage, five more, the expert offsets and tile starts, 1 KB of alignment slack)
+  using C1 = SwapCfg<GEMM1, NT, 1>;
+  constexpr int FIXED = C1::GBUF_BYTES + 5 * 8 + 16 + 8 * (kMaxExperts + 1) + 1024;
+  constexpr int STAGES = (227 * 1024 - FIXED) / (C1::STAGE + 16);
   using Cf = SwapCfg<GEMM1, NT, STAGES>;
   auto kern = swap_gemm_bf16_kernel<GEMM1, NT, STAGES>;
   static cudaError_t attr =

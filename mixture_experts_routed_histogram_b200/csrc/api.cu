@@ -110,6 +110,8 @@ moe::GemmProblem problem(const moe_shape_t& s) {
 }
 
 int* status_word(void* ws) { return reinterpret_cast<int*>(ws); }
+// K slices the decode-sized GEMM2 chose, for the combine after it (in the status region)
+int* splits_word(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 64); }
 
 template <class T>
 T* at(void* ws, size_t off) {
@@ -362,12 +364,13 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
       e = moe::launch_gemm1_swap(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
                                  part, moe::swap_splits_gemm1(p), status, stream, &n);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    int* splits_used = splits_word(ws);
     if ((e = moe::launch_gemm2_swap(p, act, offsets, static_cast<const uint16_t*>(w2), y, part,
-                                    splits, status, stream, &n)) != cudaSuccess)
+                                    splits, splits_used, status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (splits > 1) {
-      if ((e = moe::launch_combine_parts(part, splits, R, w, a2r, out, T, shape->H, k_all(*shape),
-                                         stream, &n)) != cudaSuccess)
+      if ((e = moe::launch_combine_parts(part, splits_used, R, w, a2r, out, T, shape->H,
+                                         k_all(*shape), stream, &n)) != cudaSuccess)
         return MOE_ERR_CUDA;
       g_last_launches = n;
       return MOE_OK;

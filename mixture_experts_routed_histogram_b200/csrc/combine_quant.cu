@@ -66,8 +66,9 @@ __global__ void __launch_bounds__(kCombineThreads)
 // The combine when GEMM2 split K: the k rows' partial sums are added slice by slice (in
 // slice order) before the routing weights are applied (slot order), all in fp32.
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_parts_kernel(const float* __restrict__ part, int splits, int64_t R,
-                         const float* __restrict__ w, const int32_t* __restrict__ assign2row,
+    combine_parts_kernel(const float* __restrict__ part, const int* __restrict__ splits_dev,
+                         int64_t R, const float* __restrict__ w,
+                         const int32_t* __restrict__ assign2row,
                          uint16_t* __restrict__ out, int H, int k) {
   __shared__ float sw[kMaxTopK];
   __shared__ int64_t srow[kMaxTopK];
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     srow[threadIdx.x] = static_cast<int64_t>(__ldg(assign2row + t * k + threadIdx.x)) * H;
   }
   __syncthreads();
+  const int splits = *splits_dev;  // written by the GEMM2 this kernel follows
   const int64_t slice = R * H;
   for (int c = threadIdx.x * 4; c < H; c += kCombineThreads * 4) {
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -202,7 +204,7 @@ cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* ass
                   y, w, assign2row, out, H, k);
 }
 
-cudaError_t launch_combine_parts(const float* part, int splits, int64_t R, const float* w,
+cudaError_t launch_combine_parts(const float* part, const int* splits, int64_t R, const float* w,
                                  const int32_t* assign2row, uint16_t* out, int64_t T, int H,
                                  int k, cudaStream_t stream, int* launches) {
   if (T == 0) return cudaSuccess;

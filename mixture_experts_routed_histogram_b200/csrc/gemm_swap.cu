@@ -42,7 +42,8 @@ struct SwapArgs {
   int n_out;                  // I (GEMM1) or H (GEMM2)
   int K;
   int ftiles;                 // feature tiles per expert: I/64 (GEMM1) or H/128 (GEMM2)
-  int splits;                 // K slices (GEMM2)
+  int splits;                 // K slices (GEMM1); GEMM2: the most slices it may choose
+  int* splits_used;           // GEMM2 with splits > 1: the slice count it chose (for the combine)
   int b_rows;                 // weight rows per expert: 2I or H
   int64_t R;
   int inject_stall;
@@ -86,6 +87,34 @@ __device__ __forceinline__ void decode_swap(int task, const int* s_tile, int E, 
   const int rest = local - tt * per_tile;
   ft = rest / splits;
   sp = rest - ft * splits;
+}
+
+// K slices for the decode-sized GEMM2, chosen on the device from the exact count of busy
+// (expert, token tile, feature tile) tiles, so that skewed routing (fewer busy experts than
+// min(E, R)) is seen.  Cost model, fitted to the decode workload (T = 1, 8, 32, 64): tasks
+// are dealt round-robin, so the CTAs work in rounds of up to P tasks of kb/s K blocks each;
+// one CTA alone streams only about 1/(0.75 P) of HBM bandwidth, so a round with a CTAs busy
+// takes kb/s * max(1, a / (0.75 P)) block times, and every round adds about 16 more (a task
+// switch measured that costly).  Candidates keep >= 24 K blocks per slice.
+__device__ __forceinline__ int choose_gemm2_splits(int tiles, int kb, int smax, int P) {
+  const float psat = 0.75f * static_cast<float>(P);
+  int best = 1;
+  float best_cost = 3.0e38f;
+  for (int s = 1; s <= smax; ++s) {
+    if (kb % s != 0 || (s > 1 && kb / s < 24)) continue;
+    const int n = tiles * s;
+    const int full = n / P, rem = n - full * P;
+    const float len = static_cast<float>(kb / s);
+    const float cost =
+        len * (static_cast<float>(full) * fmaxf(1.0f, static_cast<float>(P) / psat) +
+               (rem ? fmaxf(1.0f, static_cast<float>(rem) / psat) : 0.0f)) +
+        16.0f * static_cast<float>(full + (rem ? 1 : 0));
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 __device__ __forceinline__ float silu_mul_s(float g, float u) {
@@ -136,6 +165,7 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
   volatile int* s_never = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8);
+  int* s_splits = reinterpret_cast<int*>(smem + C::MISC_OFF + 12);
   int* s_off = reinterpret_cast<int*>(smem + C::OFFS_OFF);
   int* s_tile = reinterpret_cast<int*>(smem + C::TILE_OFF);
 
@@ -143,7 +173,6 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int E = args.E;
   const uint64_t lim = args.wait_limit_ns;
-  const int per_tile = args.ftiles * args.splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -193,15 +222,25 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
         run += (s_off[e + 1] - s_off[e] + NT - 1) / NT;
       }
     }
-    if (lane == 31) s_tile[E] = incl;
+    if (lane == 31) {
+      s_tile[E] = incl;
+      // args.splits > 1 selects the partial-sum output; GEMM2 picks its own slice count
+      *s_splits = (!GEMM1 && args.splits > 1)
+                      ? choose_gemm2_splits(incl * args.ftiles, args.K / BK, args.splits,
+                                            gridDim.x)
+                      : args.splits;
+      if (!GEMM1 && args.splits_used && blockIdx.x == 0) *args.splits_used = *s_splits;
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = s_tile[E] * per_tile;
   const int kb_all = args.K / BK;
-  const int kb_per = kb_all / args.splits;
+  const int splits = *s_splits;
+  const int per_tile = args.ftiles * splits;
+  const int total = s_tile[E] * per_tile;
+  const int kb_per = kb_all / splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -210,7 +249,7 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     bool ok = true;
     for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
       int e, tt, ft, sp;
-      decode_swap(task, s_tile, E, per_tile, args.splits, e, tt, ft, sp);
+      decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
       const int row0 = s_off[e] + tt * NT;
       const int wrow = GEMM1 ? e * args.b_rows + ft * 64 : e * args.b_rows + ft * BMW;
       for (int kb = sp * kb_per; kb < (sp + 1) * kb_per; ++kb, ++fill) {
@@ -300,7 +339,7 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
       bool ok = true;
       for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
         int e, tt, ft, sp;
-        decode_swap(task, s_tile, E, per_tile, args.splits, e, tt, ft, sp);
+        decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
         const int row0 = s_off[e] + tt * NT;
         const int rows = min(NT, s_off[e + 1] - row0);
         const uint16_t* src[PER];
@@ -340,7 +379,7 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     bool ok = true;
     for (int task = blockIdx.x; task < total; task += gridDim.x) {
       int e, tt, ft, sp;
-      decode_swap(task, s_tile, E, per_tile, args.splits, e, tt, ft, sp);
+      decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
       const int row0 = s_off[e] + tt * NT;
       const int rows = min(NT, s_off[e + 1] - row0);
       const int acc = tc & 1;
@@ -504,10 +543,9 @@ int swap_token_tile(int64_t T) {
 
 bool use_swap_gemm(int64_t T) { return T <= 64; }
 
-// K slices for a decode-sized GEMM: enough (expert, feature tile, slice) tasks that the
-// last, partial wave over the SMs costs little (GEMM1 >= 6 waves; GEMM2 >= 2: its slices
-// are shorter and more of them measured slower), counting at most min(E, R) busy experts; slices divide the K blocks and keep
-// >= 8 blocks each.
+// K slices for GEMM1: enough (expert, feature tile, slice) tasks that the last, partial
+// wave over the SMs costs little (>= 6 waves), counting at most min(E, R) busy experts;
+// slices divide the K blocks and keep >= 8 blocks each.
 static int splits_for(int64_t busy_tiles, int kb, int waves) {
   int best = 1;
   for (int s = 1; s <= std::min(kb, kMaxSplits); ++s) {
@@ -518,8 +556,14 @@ static int splits_for(int64_t busy_tiles, int kb, int waves) {
   return best;
 }
 
+// GEMM2: the most K slices its kernel may choose (it picks the count on the device from
+// the busy tiles): the largest divisor of the K blocks that keeps >= 24 blocks per slice.
 int swap_splits(const GemmProblem& p) {
-  return splits_for(std::min<int64_t>(p.E, p.R) * (p.H / BMW), p.I / BK, 2);
+  const int kb = p.I / BK;
+  int best = 1;
+  for (int s = 2; s <= std::min(kb, kMaxSplits); ++s)
+    if (kb % s == 0 && kb / s >= 24) best = s;
+  return best;
 }
 
 int swap_splits_gemm1(const GemmProblem& p) {
@@ -563,7 +607,8 @@ cudaError_t launch_gemm1_swap(const GemmProblem& p, const uint16_t* x, const int
 
 cudaError_t launch_gemm2_swap(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
                               const uint16_t* w2, uint16_t* y, float* part, int splits,
-                              int* status, cudaStream_t stream, int* launches) {
+                              int* splits_used, int* status, cudaStream_t stream,
+                              int* launches) {
   if (p.R == 0) return cudaSuccess;
   const int nt = swap_token_tile(p.T);
   CUtensorMap tw, tt;
@@ -581,6 +626,7 @@ cudaError_t launch_gemm2_swap(const GemmProblem& p, const uint16_t* act, const i
   a.K = p.I;
   a.ftiles = p.H / BMW;
   a.splits = splits;
+  a.splits_used = splits_used;
   a.b_rows = p.H;
   a.R = p.R;
   a.inject_stall = g_inject_stall;

@@ -93,7 +93,7 @@ cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
 // Decode-sized GEMMs with weights on the MMA's M side and token rows on its N side.
 constexpr int kMaxSplits = 16;
 bool use_swap_gemm(int64_t T);
-int swap_splits(const GemmProblem& p);        // K slices of GEMM2
+int swap_splits(const GemmProblem& p);        // the most K slices GEMM2 may choose
 int swap_splits_gemm1(const GemmProblem& p);  // K slices of GEMM1
 // splits == 1 fuses SwiGLU; splits > 1 writes fp32 gate|up partial sums part[splits][R][2I]
 // and a second kernel finishes act = silu(g)*u.
@@ -101,12 +101,15 @@ cudaError_t launch_gemm1_swap(const GemmProblem& p, const uint16_t* x, const int
                               const int32_t* offsets, const uint16_t* w13, uint16_t* act,
                               float* part, int splits, int* status, cudaStream_t stream,
                               int* launches);
-// splits == 1 writes y (bf16); splits > 1 writes fp32 partial sums part[splits][R][H].
+// splits == 1 writes y (bf16); splits > 1 writes fp32 partial sums part[S][R][H] for the
+// S <= splits slices the kernel chooses from the busy tiles, and stores S in *splits_used.
 cudaError_t launch_gemm2_swap(const GemmProblem& p, const uint16_t* act, const int32_t* offsets,
                               const uint16_t* w2, uint16_t* y, float* part, int splits,
-                              int* status, cudaStream_t stream, int* launches);
-// Combine from K-split partial sums: out[t] = sum_j w[t,j] * sum_s part[s][assign2row[t,j]].
-cudaError_t launch_combine_parts(const float* part, int splits, int64_t R, const float* w,
+                              int* splits_used, int* status, cudaStream_t stream,
+                              int* launches);
+// Combine from K-split partial sums: out[t] = sum_j w[t,j] * sum_s part[s][assign2row[t,j]],
+// with the slice count S read from *splits (written by the GEMM2 before it).
+cudaError_t launch_combine_parts(const float* part, const int* splits, int64_t R, const float* w,
                                  const int32_t* assign2row, uint16_t* out, int64_t T, int H,
                                  int k, cudaStream_t stream, int* launches);
 

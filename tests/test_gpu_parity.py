@@ -34,6 +34,10 @@ SMALL = {
     # shared experts: experts E.. on every token with weight 1 (decode-sized and large)
     "shared1_t40": I.Workload("sh1", 40, 256, 128, 8, 2, n_shared=1),
     "shared2_t500": I.Workload("sh2", 500, 512, 256, 16, 4, n_shared=2),
+    # decode-sized with K split into slices: GEMM2 picks the count from its busy tiles
+    # (2 for I = 3072; 4-6 of up to 7 for I = 10752, 168 K blocks); GEMM1 splits H = 1024 in 2
+    "ksplit_i3072": I.Workload("ks2", 24, 512, 3072, 4, 2, routing="zipf"),
+    "ksplit_h1024_i10752": I.Workload("ks7", 8, 1024, 10752, 4, 2),
 }
 
 

@@ -64,7 +64,9 @@ __global__ void __launch_bounds__(kCombineThreads)
 }
 
 // The combine when GEMM2 split K: the k rows' partial sums are added slice by slice (in
-// slice order) before the routing weights are applied (slot order), all in fp32.
+// slice order) before the routing weights are applied (slot order), all in fp32.  Decode
+// batches are a few tokens, so each token's columns are spread over blockIdx.y (one 4-column
+// chunk per thread) and a slot's slice loads are all issued before the first add.
 __global__ void __launch_bounds__(kCombineThreads)
     combine_parts_kernel(const float* __restrict__ part, const int* __restrict__ splits_dev,
                          int64_t R, const float* __restrict__ w,
@@ -82,13 +84,21 @@ __global__ void __launch_bounds__(kCombineThreads)
   __syncthreads();
   const int splits = *splits_dev;  // written by the GEMM2 this kernel follows
   const int64_t slice = R * H;
-  for (int c = threadIdx.x * 4; c < H; c += kCombineThreads * 4) {
+  const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 4;
+  if (c < H) {
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     for (int j = 0; j < k; ++j) {
+      float4 v[kMaxSplits];
+#pragma unroll
+      for (int s = 0; s < kMaxSplits; ++s)
+        if (s < splits)
+          v[s] = __ldcs(reinterpret_cast<const float4*>(part + s * slice + srow[j] + c));
       float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      for (int s = 0; s < splits; ++s) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(part + s * slice + srow[j] + c));
-        y[0] += v.x; y[1] += v.y; y[2] += v.z; y[3] += v.w;
+#pragma unroll
+      for (int s = 0; s < kMaxSplits; ++s) {
+        if (s < splits) {
+          y[0] += v[s].x; y[1] += v[s].y; y[2] += v[s].z; y[3] += v[s].w;
+        }
       }
       const float wj = sw[j];
 #pragma unroll
@@ -209,8 +219,10 @@ cudaError_t launch_combine_parts(const float* part, const int* splits, int64_t R
                                  int k, cudaStream_t stream, int* launches) {
   if (T == 0) return cudaSuccess;
   ++*launches;
-  return launch_k(combine_parts_kernel, dim3(static_cast<unsigned>(T)), dim3(kCombineThreads), 0,
-                  stream, part, splits, R, w, assign2row, out, H, k);
+  const unsigned cblocks =
+      static_cast<unsigned>((H + 4 * kCombineThreads - 1) / (4 * kCombineThreads));
+  return launch_k(combine_parts_kernel, dim3(static_cast<unsigned>(T), cblocks),
+                  dim3(kCombineThreads), 0, stream, part, splits, R, w, assign2row, out, H, k);
 }
 
 cudaError_t launch_quant_x(const uint16_t* x, uint8_t* xq, float* sx, uint32_t* sxw, int64_t T,

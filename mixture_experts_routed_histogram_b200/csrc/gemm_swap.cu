@@ -472,12 +472,22 @@ __global__ void swiglu_parts_kernel(const float* __restrict__ part, int splits, 
   const int64_t r = i / I;
   const int c = static_cast<int>(i - r * I);
   const int64_t slice = R * 2 * I;
+  // every slice's loads are issued before the first add (the sum stays in slice order)
+  float2 g[kMaxSplits], u[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < splits) {
+      const float* p = part + s * slice + r * 2 * I;
+      g[s] = *reinterpret_cast<const float2*>(p + c);
+      u[s] = *reinterpret_cast<const float2*>(p + I + c);
+    }
+  }
   float g0 = 0.f, g1 = 0.f, u0 = 0.f, u1 = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* p = part + s * slice + r * 2 * I;
-    const float2 g = *reinterpret_cast<const float2*>(p + c);
-    const float2 u = *reinterpret_cast<const float2*>(p + I + c);
-    g0 += g.x; g1 += g.y; u0 += u.x; u1 += u.y;
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < splits) {
+      g0 += g[s].x; g1 += g[s].y; u0 += u[s].x; u1 += u[s].y;
+    }
   }
   *reinterpret_cast<uint32_t*>(act + r * I + c) = pack_bf16x2(silu_mul_s(g0, u0), silu_mul_s(g1, u1));
 }

@@ -217,6 +217,20 @@ MOE_API const char *moe_status_string(moe_status_t status);
 MOE_API void moe_debug_set_wait_limit_ns(uint64_t ns);
 MOE_API void moe_debug_inject_stall(int on);
 
+/* Per-stage timing of moe_forward (host), for the per-kernel breakdown of a benchmark.
+ * After moe_debug_time_stages(1), every moe_forward call on this host thread records a
+ * CUDA event (owned by the library) on its stream before its first launch and after each
+ * stage: "route_permute" (the fused small-batch kernel) or "route" and "permute" (three
+ * kernels), "quantize_x" (FP8 x MXFP4), "gemm1_swiglu" (with the decode-sized K-split
+ * finish), "gemm2" and "combine".  The events take away the overlap that programmatic
+ * dependent launch gives consecutive kernels, so time whole steps with it off, and do not
+ * turn it on while capturing a CUDA graph.  moe_debug_stage_times waits for the last
+ * forward's final event, writes up to `max` stage names (static strings) and times in
+ * milliseconds, and returns the number of stages that forward recorded (0 if none, -1 on
+ * a CUDA error).  moe_debug_time_stages(0) turns recording off. */
+MOE_API void moe_debug_time_stages(int on);
+MOE_API int moe_debug_stage_times(const char **names, float *ms, int max);
+
 /* Number of kernel launches the last successful call of each entry point enqueued on
  * this host thread (host). */
 MOE_API int moe_last_launch_count(void);

@@ -36,7 +36,8 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute
            "moe_quantize_x", "moe_quantize_weights_mxfp4", "moe_grouped_gemm1_swiglu",
            "moe_grouped_gemm2", "moe_combine", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_debug_set_wait_limit_ns", "moe_debug_inject_stall",
-           "moe_last_launch_count", "moe_permute_noalloc")
+           "moe_last_launch_count", "moe_permute_noalloc", "moe_debug_time_stages",
+           "moe_debug_stage_times")
 
 
 class MoeShape(ctypes.Structure):
@@ -102,6 +103,10 @@ def load():
             L.moe_debug_set_wait_limit_ns.restype = None
             L.moe_debug_inject_stall.argtypes = [ctypes.c_int]; L.moe_debug_inject_stall.restype = None
             L.moe_last_launch_count.argtypes = []; L.moe_last_launch_count.restype = ctypes.c_int
+            L.moe_debug_time_stages.argtypes = [ctypes.c_int]; L.moe_debug_time_stages.restype = None
+            L.moe_debug_stage_times.argtypes = [ctypes.POINTER(ctypes.c_char_p),
+                                                ctypes.POINTER(ctypes.c_float), ctypes.c_int]
+            L.moe_debug_stage_times.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -222,3 +227,17 @@ def moe_debug_set_wait_limit_ns(ns: int):
 
 def moe_debug_inject_stall(on: bool):
     load().moe_debug_inject_stall(int(bool(on)))
+
+
+def moe_debug_time_stages(on: bool):
+    load().moe_debug_time_stages(int(bool(on)))
+
+
+def moe_debug_stage_times(max_stages: int = 8):
+    """[(stage name, ms)] of the last moe_forward recorded on this thread."""
+    names = (ctypes.c_char_p * max_stages)()
+    ms = (ctypes.c_float * max_stages)()
+    n = load().moe_debug_stage_times(names, ms, max_stages)
+    if n < 0:
+        raise MoeError(MOE_ERR_CUDA, "moe_debug_stage_times")
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n, max_stages))]

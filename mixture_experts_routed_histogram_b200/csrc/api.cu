@@ -12,6 +12,32 @@
 namespace {
 
 thread_local int g_last_launches = 0;
+
+// Per-stage timing of moe_forward (moe_debug_time_stages): an event before the first launch
+// and one after each stage, on the forward's stream.
+constexpr int kMaxTimedStages = 8;
+struct StageTimer {
+  bool on = false;
+  cudaEvent_t ev[kMaxTimedStages + 1] = {};
+  const char* name[kMaxTimedStages] = {};
+  int n = -1;  // stages recorded by the last forward (-1: none)
+  void begin(cudaStream_t st) {
+    n = -1;
+    if (!on) return;
+    for (cudaEvent_t& e : ev)
+      if (!e && cudaEventCreate(&e) != cudaSuccess) return;
+    if (cudaEventRecord(ev[0], st) == cudaSuccess) n = 0;
+  }
+  void mark(cudaStream_t st, const char* what) {
+    if (n < 0 || n >= kMaxTimedStages) return;
+    if (cudaEventRecord(ev[n + 1], st) != cudaSuccess) {
+      n = -1;
+      return;
+    }
+    name[n++] = what;
+  }
+};
+thread_local StageTimer g_timer;
 uint64_t g_wait_limit_ns = 4000000000ull;  // 4 s per bounded device wait
 
 constexpr size_t kAlign = 256;
@@ -296,6 +322,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
                          const uint8_t* w2_sf, uint16_t* out, int32_t* ids_out, void* ws,
                          size_t ws_bytes, cudaStream_t stream) {
   g_last_launches = 0;
+  g_timer.n = -1;
   MOE_TRY(check_shape(shape));
   if (!ws) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_MISALIGNED;
@@ -323,20 +350,24 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
   const moe::GemmProblem p = problem(*shape);
   int n = 0;
   cudaError_t e;
+  g_timer.begin(stream);
   if (moe::use_route_permute_small(T, e_all(*shape), k_all(*shape))) {
     if ((e = moe::launch_route_permute_small(logits, T, shape->E, shape->k, shape->n_shared,
                                              shape->score,
                                              shape->renormalize, ids, w, counts, offsets, r2a,
                                              a2r, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "route_permute");
   } else {
     if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->n_shared,
                                shape->score,
                                shape->renormalize, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "route");
     if ((e = moe::launch_permute(ids, T, k_all(*shape), e_all(*shape), counts, offsets, r2a, a2r,
                                  at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "permute");
   }
   if (fp8) {
     uint8_t* xq = at<uint8_t>(ws, L.xq);
@@ -346,12 +377,15 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     if ((e = moe::launch_quant_x(x, xq, at<float>(ws, L.sx), sxw, T, shape->H, stream, &n)) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "quantize_x");
     if ((e = moe::launch_gemm1_mx(p, xq, sxw, r2a, offsets, static_cast<const uint8_t*>(w13),
                                   w13_sf, aq, nullptr, asw, status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm1_swiglu");
     if ((e = moe::launch_gemm2_mx(p, aq, asw, offsets, static_cast<const uint8_t*>(w2), w2_sf, y,
                                   status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm2");
   } else if (moe::use_swap_gemm(T) && shape->H % 128 == 0) {
     // decode-sized: weights on the MMA's M side; GEMM2 splits K and the combine adds the
     // partial sums.  (GEMM1 with ReLU2 runs on the single-SM kernel.)
@@ -364,14 +398,17 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
       e = moe::launch_gemm1_swap(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
                                  part, moe::swap_splits_gemm1(p), status, stream, &n);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm1_swiglu");
     int* splits_used = splits_word(ws);
     if ((e = moe::launch_gemm2_swap(p, act, offsets, static_cast<const uint16_t*>(w2), y, part,
                                     splits, splits_used, status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm2");
     if (splits > 1) {
       if ((e = moe::launch_combine_parts(part, splits_used, R, w, a2r, out, T, shape->H,
                                          k_all(*shape), stream, &n)) != cudaSuccess)
         return MOE_ERR_CUDA;
+      g_timer.mark(stream, "combine");
       g_last_launches = n;
       return MOE_OK;
     }
@@ -379,13 +416,16 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     if ((e = moe::launch_gemm1_bf16(p, x, r2a, offsets, static_cast<const uint16_t*>(w13), act,
                                     status, stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm1_swiglu");
     if ((e = moe::launch_gemm2_bf16(p, act, offsets, static_cast<const uint16_t*>(w2), y, status,
                                     stream, &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    g_timer.mark(stream, "gemm2");
   }
   if ((e = moe::launch_combine(y, w, a2r, out, T, shape->H, k_all(*shape), stream, &n)) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
+  g_timer.mark(stream, "combine");
   g_last_launches = n;
   return MOE_OK;
 }
@@ -421,5 +461,21 @@ int moe_last_launch_count(void) { return g_last_launches; }
 void moe_debug_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 4000000000ull; }
 
 void moe_debug_inject_stall(int on) { moe::g_inject_stall = on ? 1 : 0; }
+
+void moe_debug_time_stages(int on) {
+  g_timer.on = on != 0;
+  g_timer.n = -1;
+}
+
+int moe_debug_stage_times(const char** names, float* ms, int max) {
+  const int n = g_timer.n;
+  if (n <= 0) return 0;
+  if (cudaEventSynchronize(g_timer.ev[n]) != cudaSuccess) return -1;
+  for (int i = 0; i < n && i < max; ++i) {
+    if (cudaEventElapsedTime(&ms[i], g_timer.ev[i], g_timer.ev[i + 1]) != cudaSuccess) return -1;
+    names[i] = g_timer.name[i];
+  }
+  return n;
+}
 
 }  // extern "C"

@@ -100,22 +100,70 @@ def max_over_ranks(v: float, world: int) -> float:
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and throttle reasons sampled while the timed region runs: NVML polled every
+    10 ms from a thread (read-only queries), else nvidia-smi's own sampling loop."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []       # (host arrival time, csv line)
+        self.nvml = None
+        self.stop = threading.Event()
+        self.lines = []       # (host arrival time, csv line) from nvidia-smi
+        self.samples = []     # (host time, sm MHz, max sm MHz, [reason names]) from NVML
         self.window = None    # (t0, t1) of the timed region
 
+    def _physical(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        if 0 <= self.index < len(vis) and vis[self.index].strip():
+            return vis[self.index].strip()
+        return str(self.index)
+
+    def _nvml_start(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            dev = self._physical()
+            h = (N.nvmlDeviceGetHandleByUUID(dev) if dev.startswith(("GPU-", "MIG-"))
+                 else N.nvmlDeviceGetHandleByIndex(int(dev)))
+            mx = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+            bits = [N.nvmlClocksEventReasonHwSlowdown, N.nvmlClocksEventReasonHwThermalSlowdown,
+                    N.nvmlClocksEventReasonSwThermalSlowdown, N.nvmlClocksEventReasonSwPowerCap]
+        except Exception:   # no NVML here: fall back to nvidia-smi
+            return False
+
+        def poll():
+            while not self.stop.is_set():
+                try:
+                    sm = float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                    r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                self.samples.append((time.time(), sm, mx,
+                                     [n for n, b in zip(self.NAMES, bits) if r & b]))
+                self.stop.wait(0.01)
+            try:
+                N.nvmlShutdown()
+            except Exception:
+                pass
+
+        self.nvml = threading.Thread(target=poll, daemon=True)
+        self.nvml.start()
+        return True
+
     def __enter__(self):
+        if self._nvml_start():
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0:   # first sample is in
+                time.sleep(0.005)
+            return self
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                ["nvidia-smi", f"--id={self._physical()}", f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
@@ -135,6 +183,9 @@ class ClockSampler:
         self.window = (t0, t1)
 
     def __exit__(self, *a):
+        self.stop.set()
+        if self.nvml is not None:
+            self.nvml.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -143,33 +194,38 @@ class ClockSampler:
                 self.proc.kill()
             self.t.join(timeout=2)
 
+    def _in_window(self, rows, slack):
+        if self.window is None:
+            return rows
+        inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1] + slack]
+        return inside if inside else rows[-2:]
+
     def summary(self):
-        if not self.lines:
-            return None
         sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = self.lines
-        if self.window is not None:
-            inside = [ln for t, ln in lines if self.window[0] <= t <= self.window[1] + 0.15]
-            lines = inside if inside else [ln for _, ln in lines[-2:]]
+        if self.samples:
+            for _, f, m, rs in self._in_window(self.samples, 0.0):
+                sm.append(f)
+                mx = max(mx, m)
+                reasons.update(rs)
+            src = "nvml, 10 ms"
         else:
-            lines = [ln for _, ln in lines]
-        for ln in lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
+            src = "nvidia-smi"
+            for _, ln in self._in_window(self.lines, 0.15):
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = max(mx, float(f[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(self.NAMES, f[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": src}
 
 
 # ---------------------------------------------------------------- workload set-up

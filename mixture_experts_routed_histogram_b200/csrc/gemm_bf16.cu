@@ -577,7 +577,7 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
   if (use_swap_gemm(p.T) && p.H % 128 == 0)
     return launch_gemm2_swap(p, act, offsets, w2, y, nullptr, 1, nullptr, status, stream,
                              launches);
-  if (use_pair_gemm(p.R, p.E))
+  if (use_pair_gemm(p.R, p.E, p.I))
     return launch_gemm2_bf16_2sm(p, act, offsets, w2, y, status, stream, launches);
   constexpr int bn = 256;
   CUtensorMap ta, tb;

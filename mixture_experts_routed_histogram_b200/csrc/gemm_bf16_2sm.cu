@@ -463,10 +463,12 @@ cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
 
 // Which grouped GEMMs run on SM pairs.  The pair kernels run their padded work about 10 %
 // faster than the single-SM ones (half the B bytes per SM), but their 256-row tiles pad
-// more rows: at ~500 rows per expert 20 % against 11 %, a wash in time and more energy
-// under the power cap.  So GEMM2 (contiguous A by TMA) pairs only once an expert averages
-// >= 768 rows, and GEMM1 (whose gathered A reaches the leader through a relay warp) stays
-// on single SMs.  MOE_PAIR_GEMM=0/1 forces the choice for both (a tuning and test switch).
+// more rows: at ~500 rows per expert 20 % against 11 %.  So GEMM2 (contiguous A by TMA)
+// pairs once an expert averages >= 768 rows, or >= 384 when its K is short (<= 1024: the
+// deeper ring of the pair kernel then pays; measured at 512 rows per expert: K = 768
+// 203 -> 198 us, K = 8192 587 -> 603 us), and GEMM1 (whose gathered A reaches the leader
+// through a relay warp) stays on single SMs (measured slower on pairs at 512-4096 rows
+// per expert).  MOE_PAIR_GEMM=0/1 forces the choice for both (a tuning and test switch).
 int pair_gemm_override() {
   static const int force = [] {
     const char* e = getenv("MOE_PAIR_GEMM");
@@ -475,9 +477,10 @@ int pair_gemm_override() {
   return force;
 }
 
-bool use_pair_gemm(int64_t R, int E) {
+bool use_pair_gemm(int64_t R, int E, int K) {
   if (pair_gemm_override() >= 0) return pair_gemm_override() != 0;
-  return R >= static_cast<int64_t>(E) * 768;
+  const int64_t per_expert = R / E;
+  return per_expert >= 768 || (K <= 1024 && per_expert >= 384);
 }
 
 bool use_pair_gemm1(int64_t R, int E) {

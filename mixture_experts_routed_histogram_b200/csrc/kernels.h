@@ -79,8 +79,8 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
                               int* launches);
 
 // The same BF16 GEMMs on SM pairs (cta_group::2, 256-row tiles); use_pair_gemm decides
-// from the average rows per expert.
-bool use_pair_gemm(int64_t R, int E);
+// for GEMM2 from the average rows per expert and its K.
+bool use_pair_gemm(int64_t R, int E, int K);
 bool use_pair_gemm1(int64_t R, int E);
 cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
                                   const int32_t* row2assign, const int32_t* offsets,

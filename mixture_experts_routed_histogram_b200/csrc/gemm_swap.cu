@@ -9,13 +9,16 @@
 //
 // Per task: 128 weight rows x NT token rows, K streamed through a STAGES-deep ring of
 // (16 KB weight box + NT*128 B token box) stages -- almost all of shared memory holds
-// weights, so each SM keeps ~150 KB of weight bytes in flight.
+// weights, so each SM keeps ~170 KB of weight bytes in flight.
 //   GEMM1: the 128 weight rows are 64 gate rows and the 64 matching up rows; the epilogue
 //          passes the gate half through shared memory to the warps that hold the up half,
-//          which write act = silu(g)*u for the tile's 64 features of each token row.
+//          which write act = silu(g)*u for the tile's 64 features of each token row.  With
+//          K split (slice count set on the host), it writes fp32 gate|up partial sums and
+//          swiglu_parts_kernel finishes act.
 //   GEMM2: 128 output features; K (= I) may be split into S slices whose fp32 partial sums
 //          go to a workspace that the split-aware combine adds up, so that even one token
-//          (two experts) spreads its weights over every SM.
+//          (two experts) spreads its weights over every SM.  S is chosen in the kernel from
+//          the busy tiles (choose_gemm2_splits) and stored for the combine.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/moe.h: host-side argument checks, workspace
 // carving and the ordering of the kernels on the caller's stream.  No allocation, no
-// synchronisation (except moe_get_device_status, which exists to synchronise).
+// synchronisation (except moe_get_device_status and moe_debug_stage_times, which exist to
+// synchronise; the optional per-stage timing creates its CUDA events once per thread).
 #include <stdint.h>
 #include <stdlib.h>
 

@@ -4,7 +4,8 @@
 One step = one full forward pass (route -> histogram/prefix-sum/permute -> GEMM1+SwiGLU ->
 GEMM2 -> combine) over one synthetic batch.  Default workload: the Qwen3-30B-A3B-shaped
 BF16 layer at T=8192 (H=2048, E=128, k=8, I=768).  Metric: routed-expert TFLOP/s
-(6*T*k*H*I per step); decode workloads also report us/layer and GB/s.
+(2*R*H*(2I + I) per step with SwiGLU, 2*R*H*(I + I) with ReLU2; R = T*(k + shared
+experts)); decode workloads also report us/layer and GB/s.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--T T]
   python bench.py --impl reference ...     # the CPU oracle on the host cores
@@ -34,9 +35,9 @@ from mixture_experts_routed_histogram_b200 import _capi as C  # noqa: E402
 from mixture_experts_routed_histogram_b200 import inputs as I  # noqa: E402
 
 METRIC = "routed MoE MLP fwd TFLOP/s on 1 B200 at T=8192; µs/layer at decode T"
-# Liger-Kernel PR #1463 benchmark table: Qwen3-30B-A3B-shaped BF16 routed-MoE forward,
-# T=8192, 1 GPU: 599.60 TFLOP/s on B300 (354.38 on H200).  Context only.
-PUBLISHED = {"qwen3_30b_a3b": 599.60}
+# Liger-Kernel PR #1463 benchmark table, BF16 routed-MoE forward at T=8192 on 1 GPU (B300;
+# the H200 figures are 354.38 and 511.36).  Context only.
+PUBLISHED = {"qwen3_30b_a3b": 599.60, "llama4_scout": 977.74}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernels, from the ncu captures summarised in profiles/ (the DRAM-bytes pass of

@@ -101,6 +101,26 @@ typedef struct {
  * invalid shape.  Sizes grow linearly in T*k*(H+I). */
 MOE_API size_t moe_workspace_size(const moe_shape_t *shape);
 
+/* Regions of the workspace in which moe_forward leaves the routing metadata of its last
+ * call: the top-k ids (only when moe_forward's ids_out is NULL) and weights [T][k], the
+ * per-expert counts [E] and offsets [E+1], and the expert-sorted permutation row2assign
+ * and assign2row [R] (int32, except MOE_WS_W which is fp32).  They let a caller inspect
+ * what the forward pass routed without running the stage entry points a second time; the
+ * layout is the forward pass's (FlashInfer PR #5129 "sorted I/O": the permutation of the
+ * expert-sorted row space).  On success *offset receives the region's byte offset from
+ * the workspace base (a multiple of 256) and *bytes its size (host pointers).  Returns
+ * MOE_ERR_INVALID_ARG for a bad shape, region or null pointer.  No device work. */
+typedef enum {
+  MOE_WS_IDS = 0,
+  MOE_WS_W = 1,
+  MOE_WS_COUNTS = 2,
+  MOE_WS_OFFSETS = 3,
+  MOE_WS_ROW2ASSIGN = 4,
+  MOE_WS_ASSIGN2ROW = 5
+} moe_ws_region_t;
+MOE_API moe_status_t moe_workspace_region(const moe_shape_t *shape, int32_t region,
+                                          size_t *offset, size_t *bytes);
+
 /* Zero the status block of a workspace (call once after allocating it). */
 MOE_API moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -131,10 +151,13 @@ MOE_API moe_status_t moe_permute(const moe_shape_t *shape, const int32_t *ids, i
  * Same inputs, outputs and results as moe_permute, bit for bit.  The per-chunk
  * histograms and their scans live in a 512 KB file-scope device array instead of the
  * workspace; it needs (2 * nch + 1) * E <= 131072 ints, where nch = ceil(T / 64) up to
- * T = 8192 and 128 beyond (the chunks grow), so every T works for E <= 510.  Larger
- * problems return MOE_ERR_UNSUPPORTED_SHAPE without launching anything.  The first call on each device
- * looks up the array's device address (cudaGetSymbolAddress, with that device current);
- * make that first call before any stream capture.  Every call shares the array: calls
+ * T = 8192 and 128 beyond (the chunks grow), so every T works for E <= 510, where E
+ * counts the shared experts (E + n_shared).  Larger problems return
+ * MOE_ERR_UNSUPPORTED_SHAPE without launching anything.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device current)
+ * and caches it with the id of the current context; the first call in a new context
+ * (for example after cudaDeviceReset) looks it up again.  Make that first call before
+ * any stream capture.  Every call shares the array: calls
  * whose kernels overlap on the GPU (other streams, other host threads) race on it;
  * calls ordered on one stream are safe, and no state carries over between them.  Ids
  * outside [0, E) are skipped, as in moe_permute, but there is no status word to record
@@ -203,7 +226,9 @@ MOE_API moe_status_t moe_forward(const moe_shape_t *shape, const uint16_t *x, co
                          size_t ws_bytes, cudaStream_t stream);
 
 /* Synchronise `stream`, read the workspace status word, clear it, and return it
- * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */
+ * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX).  A non-OK status also
+ * resets the rest of the 256-byte status block (the front end's grid-barrier words), so
+ * the workspace is usable again without moe_workspace_init. */
 MOE_API moe_status_t moe_get_device_status(void *ws, cudaStream_t stream);
 
 /* Static string for a status code (host). */
@@ -213,16 +238,19 @@ MOE_API const char *moe_status_string(moe_status_t status);
  * every device-side wait (default 4 s; 0 restores the default).  moe_debug_inject_stall(1)
  * makes CTA 0 of every following grouped-GEMM launch leave its first pipeline stage
  * unfilled, so that its consumer's bounded wait expires, the kernel unwinds and the status
- * word reads MOE_ERR_DEVICE_TIMEOUT; outputs of such calls are undefined.  (0 = off.) */
+ * word reads MOE_ERR_DEVICE_TIMEOUT; outputs of such calls are undefined.  It also makes
+ * the grid-wide barrier of moe_forward's large-batch front end (routing and permutation in
+ * one launch) wait for one arrival more than there are CTAs, with the same outcome.
+ * (0 = off.) */
 MOE_API void moe_debug_set_wait_limit_ns(uint64_t ns);
 MOE_API void moe_debug_inject_stall(int on);
 
 /* Per-stage timing of moe_forward (host), for the per-kernel breakdown of a benchmark.
  * After moe_debug_time_stages(1), every moe_forward call on this host thread records a
  * CUDA event (owned by the library) on its stream before its first launch and after each
- * stage: "route_permute" (the fused small-batch kernel) or "route" and "permute" (three
- * kernels), "quantize_x" (FP8 x MXFP4), "gemm1_swiglu" (with the decode-sized K-split
- * finish), "gemm2" and "combine".  The events take away the overlap that programmatic
+ * stage: "route_permute" (routing and permutation, one launch at every batch size),
+ * "quantize_x" (FP8 x MXFP4), "gemm1_swiglu" (with the decode-sized K-split finish),
+ * "gemm2" and "combine".  The events take away the overlap that programmatic
  * dependent launch gives consecutive kernels, so time whole steps with it off, and do not
  * turn it on while capturing a CUDA graph.  moe_debug_stage_times waits for the last
  * forward's final event, writes up to `max` stage names (static strings) and times in

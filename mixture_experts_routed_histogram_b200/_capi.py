@@ -37,7 +37,10 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute
            "moe_grouped_gemm2", "moe_combine", "moe_forward", "moe_get_device_status",
            "moe_status_string", "moe_debug_set_wait_limit_ns", "moe_debug_inject_stall",
            "moe_last_launch_count", "moe_permute_noalloc", "moe_debug_time_stages",
-           "moe_debug_stage_times")
+           "moe_debug_stage_times", "moe_workspace_region")
+
+# moe_ws_region_t
+MOE_WS_IDS, MOE_WS_W, MOE_WS_COUNTS, MOE_WS_OFFSETS, MOE_WS_ROW2ASSIGN, MOE_WS_ASSIGN2ROW = range(6)
 
 
 class MoeShape(ctypes.Structure):
@@ -83,6 +86,8 @@ def load():
             st, sz = ctypes.c_int, ctypes.c_size_t
             L.moe_workspace_size.argtypes = [S]; L.moe_workspace_size.restype = sz
             L.moe_workspace_init.argtypes = [vp, sz, vp]; L.moe_workspace_init.restype = st
+            L.moe_workspace_region.argtypes = [S, ctypes.c_int32, P(sz), P(sz)]
+            L.moe_workspace_region.restype = st
             L.moe_route.argtypes = [S, vp, vp, vp, vp]; L.moe_route.restype = st
             L.moe_permute.argtypes = [S, vp, vp, vp, vp, vp, vp, sz, vp]; L.moe_permute.restype = st
             L.moe_permute_noalloc.argtypes = [S, vp, vp, vp, vp, vp, vp]
@@ -152,6 +157,14 @@ def moe_workspace_size(shape: MoeShape) -> int:
 
 def moe_workspace_init(ws, stream=None):
     _check(load().moe_workspace_init(_p(ws), _nbytes(ws), _s(stream)), "moe_workspace_init")
+
+
+def moe_workspace_region(shape: MoeShape, region: int):
+    """(byte offset, bytes) of one routing-metadata region of the forward's workspace."""
+    off, n = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().moe_workspace_region(ctypes.byref(shape), int(region), ctypes.byref(off),
+                                       ctypes.byref(n)), "moe_workspace_region")
+    return int(off.value), int(n.value)
 
 
 def moe_route(shape, logits, ids, w, stream=None):

@@ -102,3 +102,34 @@ def test_workspace_size_grows_with_tokens(moelib):
 def test_status_strings(moelib):
     for st in range(8):
         assert moelib.status_string(st) != "unknown status"
+
+
+@pytest.mark.parametrize("kw", [dict(T=1), dict(T=64, n_shared=1), dict(T=8192, E=128, k=8),
+                                dict(T=300, E=1000, k=32, dtype="fp8_mxfp4")])
+def test_workspace_regions_are_disjoint_and_inside(moelib, kw):
+    """The routing-metadata regions of the forward's workspace: 256-byte aligned, past the
+    status block, inside moe_workspace_size, pairwise disjoint, and of the documented size."""
+    s = _shape(moelib, **kw)
+    total = moelib.moe_workspace_size(s)
+    R, E = s.T * (s.k + s.n_shared), s.E + s.n_shared
+    want = {moelib.MOE_WS_IDS: 4 * R, moelib.MOE_WS_W: 4 * R, moelib.MOE_WS_COUNTS: 4 * E,
+            moelib.MOE_WS_OFFSETS: 4 * (E + 1), moelib.MOE_WS_ROW2ASSIGN: 4 * R,
+            moelib.MOE_WS_ASSIGN2ROW: 4 * R}
+    spans = []
+    for region, nbytes in want.items():
+        off, n = moelib.moe_workspace_region(s, region)
+        assert n == nbytes and off % 256 == 0 and off >= 256 and off + n <= total
+        spans.append((off, off + n))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+
+
+def test_workspace_region_rejects_bad_arguments(moelib):
+    L = moelib.load()
+    s = _shape(moelib)
+    off, n = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.moe_workspace_region(ctypes.byref(s), 6, ctypes.byref(off), ctypes.byref(n)) == 1
+    assert L.moe_workspace_region(ctypes.byref(s), -1, ctypes.byref(off), ctypes.byref(n)) == 1
+    assert L.moe_workspace_region(ctypes.byref(s), 0, None, ctypes.byref(n)) == 1
+    bad = _shape(moelib, k=9)
+    assert L.moe_workspace_region(ctypes.byref(bad), 0, ctypes.byref(off), ctypes.byref(n)) == 1

@@ -19,6 +19,9 @@
 //      warp with __match_any_sync and across the 8 warps with round-stamped per-warp
 //      counts, so the row of assignment a is offsets[e] + #{a' < a : ids[a'] == e}: the
 //      stable order.
+#include <cuda.h>
+
+#include <algorithm>
 #include <mutex>
 
 #include "kernels.h"
@@ -385,6 +388,269 @@ cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, in
                          row2assign, assign2row, stream);
 }
 
+// ---------------------------------------------------------------- larger batches, one launch
+//
+// The forward pass's front end for batches beyond the single-CTA kernel: routing, the
+// per-block histograms, their scan and the stable scatter in one cooperative launch (every
+// CTA is resident, so the CTAs may wait for one another), sized so that each warp routes
+// about one token: nb CTAs of 16 warps, CTA b owning tokens [b * tpc, (b+1) * tpc).
+//   phase 1  warps route their tokens (route_token_warp), write ids and w, and count the
+//            CTA's assignments per expert in shared memory -> cc[e][b];
+//   barrier  (grid-wide: an arrival count and a generation word in the workspace's status
+//            block, bounded wait)
+//   phase 2  one warp per expert scans cc[e][0..nb) -> base[e][b] (the expert's assignments
+//            in earlier blocks) and tot[e];
+//   barrier
+//   phase 3  each CTA scans tot over the experts (offsets; CTA 0 writes counts and offsets)
+//            and scatters its assignments in order with the warp-match and round-stamp
+//            ranking of scatter_kernel: row = offsets[e] + #{a' < a : ids[a'] == e}.
+// Same outputs as launch_route followed by launch_permute, bit for bit.
+
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedMaxBlocks = 1024;
+
+int fused_blocks_cap(int64_t T) {
+  return static_cast<int>(std::min<int64_t>((T + kFusedWarps - 1) / kFusedWarps, kFusedMaxBlocks));
+}
+
+// In-place exclusive scan of s[0..n) (n <= 4 * kFusedThreads); returns the total.
+__device__ int fused_exclusive_scan(int* s, int n, int* warp_sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kFusedThreads - 1) / kFusedThreads;  // <= 4
+  const int begin = tid * per;
+  int local[4];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = begin + i;
+    local[i] = (i < per && idx < n) ? s[idx] : 0;
+    sum += local[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int warp_off = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kFusedWarps; ++w) {
+    const int v = warp_sums[w];
+    if (w < warp) warp_off += v;
+    total += v;
+  }
+  int run = warp_off + incl - sum;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int idx = begin + i;
+    if (i < per && idx < n) {
+      s[idx] = run;
+      run += local[i];
+    }
+  }
+  __syncthreads();
+  return total;
+}
+
+// Grid-wide barrier of a cooperative launch: gbar[0] counts arrivals (the last one resets it
+// and advances gbar[1]); the others wait, bounded, for the generation to move.  `extra`
+// arrivals more than the grid are awaited (a test hook that makes the wait run out).
+// Returns false (every thread of the CTA) if the wait gave up.
+__device__ bool grid_barrier(unsigned* gbar, int* s_ok, uint64_t limit_ns, unsigned extra) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned* vgen = gbar + 1;
+    const unsigned gen = *vgen;
+    __threadfence();
+    bool ok = true;
+    if (atomicAdd(gbar, 1u) == gridDim.x - 1 + extra) {
+      atomicExch(gbar, 0u);
+      __threadfence();
+      atomicAdd(gbar + 1, 1u);
+    } else {
+      const uint64_t start = globaltimer_ns();
+      for (uint32_t i = 0; *vgen == gen; ++i) {
+        if ((i & 63u) == 63u && globaltimer_ns() - start > limit_ns) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(kFusedThreads)
+    route_permute_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int ns,
+                         int score, int renorm, int tpc, int32_t* __restrict__ ids,
+                         float* __restrict__ w, int32_t* __restrict__ cc,
+                         int32_t* __restrict__ base, int32_t* __restrict__ tot,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ row2assign, int32_t* __restrict__ assign2row,
+                         unsigned* gbar, int* status, uint64_t limit_ns, int inject_stall) {
+  extern __shared__ int fsm[];
+  const int Ea = E + ns, ks = k + ns;
+  const int nb = gridDim.x;
+  int* hist = fsm;                 // [Ea]: the block's histogram, later tot and its scan
+  int* cursor = hist + Ea;         // [Ea]: the block's first row per expert
+  int* wcnt = cursor + Ea;         // [kFusedWarps][Ea]: round-stamped per-warp counts
+  __shared__ int warp_sums[kFusedWarps];
+  __shared__ int s_ok;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int me = blockIdx.x;
+  const int64_t t0 = min(static_cast<int64_t>(me) * tpc, T);
+  const int64_t t1 = min(t0 + tpc, T);
+  for (int e = tid; e < Ea; e += kFusedThreads) {
+    hist[e] = 0;
+    for (int ww = 0; ww < kFusedWarps; ++ww) wcnt[ww * Ea + e] = -1;
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  __syncthreads();
+
+  // ---- phase 1: route the block's tokens, count its assignments per expert
+  for (int64_t t = t0 + warp; t < t1; t += kFusedWarps) {
+    int id;
+    float wt;
+    route_token_warp<VPT>(logits + t * E, E, k, score, renorm, lane, id, wt);
+    if (lane >= k) {
+      id = E + (lane - k);
+      wt = 1.0f;
+    }
+    if (lane < ks) {
+      ids[t * ks + lane] = id;
+      w[t * ks + lane] = wt;
+      atomicAdd(&hist[id], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < Ea; e += kFusedThreads) cc[static_cast<int64_t>(e) * nb + me] = hist[e];
+
+  bool ok = grid_barrier(gbar, &s_ok, limit_ns, inject_stall ? 1u : 0u);
+
+  // ---- phase 2: one warp per expert scans its counts over the blocks
+  if (ok) {
+    for (int e = me * kFusedWarps + warp; e < Ea; e += nb * kFusedWarps) {
+      const int32_t* src = cc + static_cast<int64_t>(e) * nb;
+      int32_t* dst = base + static_cast<int64_t>(e) * nb;
+      int run = 0;
+      for (int c0 = 0; c0 < nb; c0 += 32) {
+        const int v = c0 + lane < nb ? __ldcg(src + c0 + lane) : 0;
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        if (c0 + lane < nb) dst[c0 + lane] = run + incl - v;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) tot[e] = run;
+    }
+    ok = grid_barrier(gbar, &s_ok, limit_ns, 0u);
+  }
+  if (!ok) {
+    // a wait gave up (status recorded; outputs undefined): leave no expert any rows, so the
+    // GEMMs after this kernel read no permutation entry
+    if (tid == 0) set_status(status, kStatusTimeout);
+    for (int e = tid; e <= Ea; e += kFusedThreads) {
+      offsets[e] = 0;
+      if (e < Ea) counts[e] = 0;
+    }
+    return;
+  }
+
+  // ---- phase 3: offsets, this block's first row per expert, stable scatter
+  for (int e = tid; e < Ea; e += kFusedThreads) {
+    hist[e] = __ldcg(tot + e);
+    cursor[e] = __ldcg(base + static_cast<int64_t>(e) * nb + me);
+  }
+  __syncthreads();
+  const int grand = fused_exclusive_scan(hist, Ea, warp_sums);
+  for (int e = tid; e < Ea; e += kFusedThreads) {
+    cursor[e] += hist[e];
+    if (me == 0) {
+      offsets[e] = hist[e];
+      counts[e] = (e + 1 < Ea ? hist[e + 1] : grand) - hist[e];
+    }
+  }
+  if (me == 0 && tid == 0) offsets[Ea] = grand;
+  __syncthreads();
+  const int64_t a0 = t0 * ks, a1 = t1 * ks;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = 0; a0 + static_cast<int64_t>(r) * kFusedThreads < a1; ++r) {
+    const int64_t a = a0 + static_cast<int64_t>(r) * kFusedThreads + tid;
+    const int e = a < a1 ? __ldcg(ids + a) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt);
+    const int grp = __popc(peers);
+    const bool leader = (__ffs(peers) - 1) == lane;
+    if (e >= 0 && leader) wcnt[warp * Ea + e] = (r << 10) | grp;
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int ww = 0; ww < warp; ++ww) {
+        const int v = wcnt[ww * Ea + e];
+        if ((v >> 10) == r) before += v & 1023;
+      }
+      const int row = cursor[e] + before + rank;
+      row2assign[row] = static_cast<int32_t>(a);
+      assign2row[a] = row;
+    }
+    __syncthreads();
+    if (e >= 0 && leader) atomicAdd(&cursor[e], grp);
+  }
+}
+
+size_t route_permute_scratch_bytes(int64_t T, int E) {
+  return (static_cast<size_t>(2) * E * fused_blocks_cap(T) + E) * sizeof(int32_t);
+}
+
+template <int VPT>
+cudaError_t launch_fused(const float* logits, int64_t T, int E, int k, int ns, int score,
+                         int renorm, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                         int32_t* row2assign, int32_t* assign2row, int32_t* scratch,
+                         unsigned* gbar, int* status, uint64_t limit_ns, cudaStream_t stream) {
+  const int Ea = E + ns;
+  const size_t smem = sizeof(int) * static_cast<size_t>(Ea) * (2 + kFusedWarps);
+  auto kern = route_permute_kernel<VPT>;
+  static cudaError_t attr = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(int) * kMaxExperts * (2 + kFusedWarps));
+  if (attr != cudaSuccess) return attr;
+  // as many CTAs as can be resident (every one must be, they wait for each other), at most
+  // one per 16 tokens
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int nb = std::max(1, std::min(fused_blocks_cap(T), per_sm * num_sms()));
+  const int tpc = static_cast<int>((T + nb - 1) / nb);
+  const int nb_used = static_cast<int>((T + tpc - 1) / tpc);   // no empty CTA
+  int32_t* cc = scratch;
+  int32_t* base = cc + static_cast<int64_t>(Ea) * nb_used;
+  int32_t* tot = base + static_cast<int64_t>(Ea) * nb_used;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nb_used);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: they wait for each other
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, logits, T, E, k, ns, score, renorm, tpc, ids, w, cc, base,
+                            tot, counts, offsets, row2assign, assign2row, gbar, status, limit_ns,
+                            g_inject_stall);
+}
+
 // ---------------------------------------------------------------- allocation-free variant
 //
 // For callers that cannot hand the library a workspace: the per-chunk histograms and their
@@ -400,26 +666,84 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 namespace {
 std::mutex g_noalloc_mu;
 constexpr int kMaxDevices = 64;
-int32_t* g_noalloc_ptr[kMaxDevices] = {};
+struct NoAllocSlot {
+  unsigned long long ctx_id = 0;  // unique id of the context the address belongs to
+  int32_t* ptr = nullptr;
+};
+NoAllocSlot g_noalloc[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
+}
+
+// Process-unique id of the calling thread's current context (0: none bound yet).
+cudaError_t current_ctx_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get || !get_id) return cudaErrorInitializationError;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
+  *id = 0;
+  if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorInitializationError;
+  return cudaSuccess;
+}
 }  // namespace
 
-// Device address of g_noalloc_scratch on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device (with
-// that device current) and cached.
+// Device address of g_noalloc_scratch in the current device's context.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with the device
+// current (cudaGetSymbolAddress) and cached per device together with the id of the context
+// it was found in (ids are never reused within a process); a new context on that device,
+// after cudaDeviceReset or a primary context released and created again (the module is
+// then loaded again, possibly elsewhere), is looked up afresh.
 static cudaError_t noalloc_scratch(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned long long id = 0;
+  if ((e = current_ctx_id(&id)) != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoAllocSlot& slot = g_noalloc[dev];
+  if (!slot.ptr || id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // binds the primary context if needed
     if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+    if ((e = current_ctx_id(&id)) != cudaSuccess) return e;
+    if (id == 0) return cudaErrorInitializationError;
+    slot.ptr = static_cast<int32_t*>(p);
+    slot.ctx_id = id;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
+}
+
+cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int ns, int score,
+                                 int renorm, int32_t* ids, float* w, int32_t* counts,
+                                 int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                 int32_t* scratch, unsigned* gbar, int* status,
+                                 uint64_t limit_ns, cudaStream_t stream, int* launches) {
+  if (T == 0) return permute_empty(E + ns, counts, offsets, stream, launches);
+  ++*launches;
+  const int need = (E + 31) / 32;
+#define MOE_FUSED(V)                                                                           \
+  return launch_fused<V>(logits, T, E, k, ns, score, renorm, ids, w, counts, offsets,          \
+                         row2assign, assign2row, scratch, gbar, status, limit_ns, stream)
+  if (need <= 1) MOE_FUSED(1);
+  if (need <= 2) MOE_FUSED(2);
+  if (need <= 4) MOE_FUSED(4);
+  if (need <= 8) MOE_FUSED(8);
+  if (need <= 16) MOE_FUSED(16);
+  MOE_FUSED(32);
+#undef MOE_FUSED
 }
 
 bool permute_noalloc_fits(int64_t T, int E) {

@@ -72,7 +72,9 @@ WsLayout layout(const moe_shape_t& s) {
   L.offsets = o; o = up(o + 4 * (E + 1));
   L.r2a = o; o = up(o + 4 * R);
   L.a2r = o; o = up(o + 4 * R);
-  L.scratch = o; o = up(o + moe::permute_scratch_bytes(static_cast<int64_t>(T), e_all(s)));
+  L.scratch = o;
+  o = up(o + std::max(moe::permute_scratch_bytes(static_cast<int64_t>(T), e_all(s)),
+                      moe::route_permute_scratch_bytes(static_cast<int64_t>(T), e_all(s))));
   L.xq = o; o = up(o + (fp8 ? T * H : 0));
   L.sx = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
   L.sxw = o; o = up(o + (fp8 ? 4 * T * (H / 128) : 0));
@@ -139,6 +141,10 @@ moe::GemmProblem problem(const moe_shape_t& s) {
 int* status_word(void* ws) { return reinterpret_cast<int*>(ws); }
 // K slices the decode-sized GEMM2 chose, for the combine after it (in the status region)
 int* splits_word(void* ws) { return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 64); }
+// arrival count and generation of the front end's grid-wide barrier (in the status region)
+unsigned* grid_barrier_words(void* ws) {
+  return reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + 128);
+}
 
 template <class T>
 T* at(void* ws, size_t off) {
@@ -152,6 +158,23 @@ extern "C" {
 size_t moe_workspace_size(const moe_shape_t* shape) {
   if (check_shape(shape) != MOE_OK) return 0;
   return layout(*shape).total;
+}
+
+moe_status_t moe_workspace_region(const moe_shape_t* shape, int32_t region, size_t* offset,
+                                  size_t* bytes) {
+  if (!offset || !bytes || check_shape(shape) != MOE_OK) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = layout(*shape);
+  const size_t R = static_cast<size_t>(shape->T) * k_all(*shape), E = e_all(*shape);
+  switch (region) {
+    case MOE_WS_IDS: *offset = L.ids; *bytes = 4 * R; break;
+    case MOE_WS_W: *offset = L.w; *bytes = 4 * R; break;
+    case MOE_WS_COUNTS: *offset = L.counts; *bytes = 4 * E; break;
+    case MOE_WS_OFFSETS: *offset = L.offsets; *bytes = 4 * (E + 1); break;
+    case MOE_WS_ROW2ASSIGN: *offset = L.r2a; *bytes = 4 * R; break;
+    case MOE_WS_ASSIGN2ROW: *offset = L.a2r; *bytes = 4 * R; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
 }
 
 moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -360,15 +383,13 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
       return MOE_ERR_CUDA;
     g_timer.mark(stream, "route_permute");
   } else {
-    if ((e = moe::launch_route(logits, ids, w, T, shape->E, shape->k, shape->n_shared,
-                               shape->score,
-                               shape->renormalize, stream, &n)) != cudaSuccess)
+    if ((e = moe::launch_route_permute(logits, T, shape->E, shape->k, shape->n_shared,
+                                       shape->score, shape->renormalize, ids, w, counts,
+                                       offsets, r2a, a2r, at<int32_t>(ws, L.scratch),
+                                       grid_barrier_words(ws), status, g_wait_limit_ns, stream,
+                                       &n)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    g_timer.mark(stream, "route");
-    if ((e = moe::launch_permute(ids, T, k_all(*shape), e_all(*shape), counts, offsets, r2a, a2r,
-                                 at<int32_t>(ws, L.scratch), status, stream, &n)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    g_timer.mark(stream, "permute");
+    g_timer.mark(stream, "route_permute");
   }
   if (fp8) {
     uint8_t* xq = at<uint8_t>(ws, L.xq);
@@ -438,7 +459,9 @@ moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
   if (cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (host != 0 && cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return MOE_ERR_CUDA;
+  // after a device-side failure the whole status block (with the grid barrier's words,
+  // which a wait that gave up may leave mid-count) starts again from zero
+  if (host != 0 && cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
   return static_cast<moe_status_t>(host);
 }

@@ -533,6 +533,8 @@ cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int
   if (!relu2 && use_swap_gemm(p.T))
     return launch_gemm1_swap(p, x, row2assign, offsets, w13, act, nullptr, 1, status, stream,
                              launches);
+  if (use_pair_swap(p))
+    return launch_gemm1_pair_swap(p, x, row2assign, offsets, w13, act, status, stream, launches);
   if (!relu2 && p.I % 128 == 0 && !use_gather4() && use_pair_gemm1(p.R, p.E))
     return launch_gemm1_bf16_2sm(p, x, row2assign, offsets, w13, act, status, stream, launches);
   // SwiGLU: 128 gate + 128 up rows per tile when I % 128 == 0, else 64 + 64;
@@ -577,6 +579,8 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
   if (use_swap_gemm(p.T) && p.H % 128 == 0)
     return launch_gemm2_swap(p, act, offsets, w2, y, nullptr, 1, nullptr, status, stream,
                              launches);
+  if (use_pair_swap(p))
+    return launch_gemm2_pair_swap(p, act, offsets, w2, y, status, stream, launches);
   if (use_pair_gemm(p.R, p.E, p.I))
     return launch_gemm2_bf16_2sm(p, act, offsets, w2, y, status, stream, launches);
   constexpr int bn = 256;

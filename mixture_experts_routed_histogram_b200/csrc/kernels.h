@@ -42,6 +42,19 @@ cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, in
                                        int32_t* counts, int32_t* offsets, int32_t* row2assign,
                                        int32_t* assign2row, cudaStream_t stream, int* launches);
 
+// Routing + histogram + prefix sum + stable scatter for larger batches in one cooperative
+// launch (one CTA per chunk of launch_permute, a grid-wide barrier between the histograms
+// and the scatter).  Same outputs as launch_route followed by launch_permute.  `scratch`
+// holds the per-block histograms and their scans (route_permute_scratch_bytes); `gbar` two
+// zero-initialised words of the barrier (left zeroed by each call); a barrier wait beyond
+// limit_ns sets `status`.
+size_t route_permute_scratch_bytes(int64_t T, int E);
+cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int ns, int score,
+                                 int renorm, int32_t* ids, float* w, int32_t* counts,
+                                 int32_t* offsets, int32_t* row2assign, int32_t* assign2row,
+                                 int32_t* scratch, unsigned* gbar, int* status,
+                                 uint64_t limit_ns, cudaStream_t stream, int* launches);
+
 // Weighted top-k combine.
 cudaError_t launch_combine(const uint16_t* y, const float* w, const int32_t* assign2row,
                            uint16_t* out, int64_t T, int H, int k, cudaStream_t stream,
@@ -89,6 +102,17 @@ cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
 cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
                                   const int32_t* offsets, const uint16_t* w2, uint16_t* y,
                                   int* status, cudaStream_t stream, int* launches);
+
+// Large-batch BF16 GEMMs on SM pairs with the weights on the MMA's M = 256 side and
+// chunks of up to 256 token rows on its N side (gemm_pair_swap.cu).
+bool use_pair_swap(const GemmProblem& p);
+cudaError_t launch_gemm1_pair_swap(const GemmProblem& p, const uint16_t* x,
+                                   const int32_t* row2assign, const int32_t* offsets,
+                                   const uint16_t* w13, uint16_t* act, int* status,
+                                   cudaStream_t stream, int* launches);
+cudaError_t launch_gemm2_pair_swap(const GemmProblem& p, const uint16_t* act,
+                                   const int32_t* offsets, const uint16_t* w2, uint16_t* y,
+                                   int* status, cudaStream_t stream, int* launches);
 
 // Decode-sized GEMMs with weights on the MMA's M side and token rows on its N side.
 constexpr int kMaxSplits = 16;

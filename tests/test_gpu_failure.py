@@ -100,3 +100,35 @@ def test_injected_stall_reports_timeout_and_context_survives(case, which):
             ref = oracle.gemm2_bf16_rows(I.bits(st["a_in"]), I.bits(inp["w2"]),
                                          np.arange(wl.R), ex)
         assert_close(f64(again), ref, what=f"{which} after recovery")
+
+
+def test_front_end_barrier_timeout_and_recovery():
+    """moe_forward's large-batch front end (routing and permutation in one cooperative
+    launch) waits at a grid-wide barrier; with the hook it waits for one CTA too many, the
+    bounded wait expires, the status reads MOE_ERR_DEVICE_TIMEOUT (reading it resets the
+    barrier's words), and the next call gives the clean call's bits again."""
+    wl = I.Workload("fe", 300, 256, 128, 16, 4)
+    inp = I.make_inputs(wl, 0, dev())
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+
+    def fwd():
+        out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev())
+        C.moe_forward(shape, inp["x"], inp["logits"], inp["w13"], None, inp["w2"], None, out,
+                      None, ws)
+        torch.cuda.synchronize()
+        return out
+
+    clean = fwd()
+    assert C.moe_get_device_status(ws) == 0
+    C.moe_debug_set_wait_limit_ns(50_000_000)
+    C.moe_debug_inject_stall(True)
+    try:
+        fwd()
+        assert C.moe_get_device_status(ws) == C.MOE_ERR_DEVICE_TIMEOUT
+    finally:
+        C.moe_debug_inject_stall(False)
+        C.moe_debug_set_wait_limit_ns(0)
+    again = fwd()
+    assert C.moe_get_device_status(ws) == 0
+    assert torch.equal(again.view(torch.int16), clean.view(torch.int16))

@@ -260,3 +260,51 @@ def test_forward_full_size_parity(name):
     inp = I.make_inputs(wl, 0, dev())
     n = 64 if wl.name == "decode" else 256
     _check_forward(wl, inp, inp["logits"], I.parity_tokens(wl.T, n))
+
+
+# Expert row counts that put an expert's last token chunk (of up to 256 rows, padded to a
+# multiple of 16) on every boundary: 1, 15-17, 31-33 rows, exactly one and two chunks, one
+# row more or less, and empty experts between them.
+CHUNK_COUNTS = [1, 0, 15, 16, 17, 31, 32, 33, 0, 255, 256, 257, 511, 512, 513, 8]
+
+
+def _chunk_ids():
+    ids = np.repeat(np.arange(len(CHUNK_COUNTS), dtype=np.int32), CHUNK_COUNTS)
+    rng = np.random.default_rng(11)
+    return rng.permutation(ids).reshape(-1, 1)        # k = 1: one slot per token
+
+
+@pytest.mark.parametrize("H,Iw,act", [(256, 128, "swiglu"), (384, 192, "swiglu"),
+                                     (512, 320, "relu2")])
+def test_gemms_on_chunk_boundaries(H, Iw, act):
+    ids = _chunk_ids()
+    T, E = ids.shape[0], len(CHUNK_COUNTS)
+    wl = I.Workload("chunks", T, H, Iw, E, 1, act=act)
+    inp = I.make_inputs(wl, 0, dev())
+    oc, oo, or2a, oa2r = oracle.permute(ids, E)
+    assert list(oc) == CHUNK_COUNTS
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    R = wl.R
+    buf, act_t = with_canary(R, Iw)
+    C.moe_grouped_gemm1_swiglu(shape, inp["x"], None, to_dev_i32(or2a), to_dev_i32(oo),
+                               inp["w13"], None, act_t, None, ws)
+    buf2, y = with_canary(R, H)
+    g = torch.Generator(device=dev()).manual_seed(5)
+    a2 = torch.randn(R, Iw, generator=g, device=dev()).to(torch.bfloat16)
+    C.moe_grouped_gemm2(shape, a2, None, to_dev_i32(oo), inp["w2"], None, y, ws)
+    torch.cuda.synchronize()
+    assert C.moe_get_device_status(ws) == 0
+    assert canary_intact(buf, R, Iw) and canary_intact(buf2, R, H)
+    tok = or2a.astype(np.int64)
+    ex = np.repeat(np.arange(E), np.diff(oo)).astype(np.int32)
+    ref1 = oracle.gemm1_bf16_rows(I.bits(inp["x"]), I.bits(inp["w13"]), tok, ex, act=act)
+    assert_close(f64(act_t), ref1, what=f"gemm1 chunks {act}")
+    ref2 = oracle.gemm2_bf16_rows(I.bits(a2), I.bits(inp["w2"]), np.arange(R), ex)
+    assert_close(f64(y), ref2, what="gemm2 chunks")
+    # every row separately: a tile that wrote another expert's rows would show here
+    got1 = f64(act_t)
+    for e in range(E):
+        lo, hi = oo[e], oo[e + 1]
+        if hi > lo:
+            assert_close(got1[lo:hi], ref1[lo:hi], what=f"gemm1 expert {e}")

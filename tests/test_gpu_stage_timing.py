@@ -1,6 +1,6 @@
 """moe_debug_time_stages: the events moe_forward records name every stage of the path the
-shape takes (fused small-batch front end or route + permute; FP8 quantisation; K-split
-decode GEMMs), each stage takes positive time, the output is the same bits as an untimed
+shape takes (the front end -- routing and permutation in one launch at every batch size;
+FP8 quantisation; K-split decode GEMMs), each stage takes positive time, the output is the same bits as an untimed
 forward, and turning it off stops the recording."""
 import pytest
 import torch
@@ -16,9 +16,9 @@ CASES = {
     "ksplit_decode": (I.Workload("ks", 24, 512, 3072, 4, 2, routing="zipf"),
                       ["route_permute", "gemm1_swiglu", "gemm2", "combine"]),
     "bf16_many_tiles": (I.Workload("m", 1000, 512, 256, 8, 4),
-                        ["route", "permute", "gemm1_swiglu", "gemm2", "combine"]),
+                        ["route_permute", "gemm1_swiglu", "gemm2", "combine"]),
     "fp8": (I.Workload("f8", 300, 256, 256, 4, 2, dtype="fp8_mxfp4"),
-            ["route", "permute", "quantize_x", "gemm1_swiglu", "gemm2", "combine"]),
+            ["route_permute", "quantize_x", "gemm1_swiglu", "gemm2", "combine"]),
 }
 
 

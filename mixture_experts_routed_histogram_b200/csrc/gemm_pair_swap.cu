@@ -33,11 +33,11 @@
 // Weight rows past the expert's own (a ragged last feature tile) read the next expert's
 // rows or the tensor map's zero fill; their outputs are never stored.
 //
-// Roles per CTA: warp 0 TMA producer (weights; GEMM2 also the token rows, as up to five
-// boxes of 128/64/32/16/8 rows), warp 1 TMEM owner and, in the leader CTA, the MMA issuer,
+// Roles per CTA: warp 0 TMA producer (weights; GEMM2 also the token rows, one 128-row box
+// per stage), warp 1 TMEM owner and, in the leader CTA, the MMA issuer,
 // warps 2-5 epilogue, and for GEMM1 warps 6-9 gather the token rows of x with 16-byte
 // cp.async and warp 10 relays "this CTA's rows of the stage have landed" to the leader.
-// Pair protocol (as gemm_bf16_2sm.cu): full[s] lives in the leader and counts both CTAs'
+// Pair protocol: full[s] lives in the leader and counts both CTAs'
 // TMA bytes (one expect-tx arrival by the leader) plus, for GEMM1, one relay arrival per
 // CTA; the leader's commits multicast to both CTAs' empty[s] and tfull[acc]; tempty[acc]
 // in the leader takes one arrival per epilogue warp of either CTA.  Every wait is bounded;
@@ -50,8 +50,6 @@
 // one TMA tensor store writes out when all 32 rows belong to the chunk (else row by row, so
 // the next expert's rows are never touched).
 #include <cudaTypedefs.h>
-
-#include <stdlib.h>
 
 #include <mutex>
 
@@ -68,7 +66,6 @@ constexpr int kHalf = kChunk / 2;
 constexpr int WROWS = 128;       // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kLoaderWarps = 4;
 constexpr int kRelayWarp = 6 + kLoaderWarps;
-constexpr int kTokBoxes = 5;     // token-row boxes of 128, 64, 32, 16 and 8 rows (GEMM2)
 
 enum Mode : int { kSwiGLU = 0, kReLU2 = 1, kGemm2 = 2 };
 
@@ -85,10 +82,6 @@ struct PsArgs {
   int b_rows;                  // weight rows per expert: 2I, I (ReLU2) or H
   int inject_stall;
   uint64_t wait_limit_ns;
-};
-
-struct TokMaps {
-  CUtensorMap m[kTokBoxes];    // act [R][I] with boxes of 128 >> i rows (GEMM2)
 };
 
 template <int MODE, int STAGES>
@@ -248,7 +241,7 @@ __device__ __forceinline__ void epi_block(uint32_t tq, uint32_t buf, int lane) {
 template <int MODE, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PsCfg<MODE, STAGES>::THREADS, 1)
     pair_swap_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
-                          const __grid_constant__ TokMaps tmT,
+                          const __grid_constant__ CUtensorMap tmT,
                           const __grid_constant__ CUtensorMap tmO, const PsArgs args) {
   using C = PsCfg<MODE, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -291,8 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PsCfg<MODE, STAGES>:
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW);
-    if constexpr (MODE == kGemm2)
-      for (int i = 0; i < kTokBoxes; ++i) tma_prefetch_desc(&tmT.m[i]);
+    if constexpr (MODE == kGemm2) tma_prefetch_desc(&tmT);
   }
   if (warp == 1) {
     tmem_alloc_2sm(s_tmem, C::TMEM_COLS);
@@ -375,28 +367,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PsCfg<MODE, STAGES>:
         const uint32_t fb = full_leader0 + 8u * static_cast<uint32_t>(s);
         if (lane == 0) {
           if (rank == 0)
-            mbar_arrive_expect_tx(&full[s], MODE == kGemm2
-                                                ? 2 * C::A_BYTES + c.n * BK * 2
-                                                : 2 * C::A_BYTES);
+            mbar_arrive_expect_tx(&full[s], MODE == kGemm2 ? 2 * C::STAGE : 2 * C::A_BYTES);
           if constexpr (MODE == kSwiGLU) {
             // four blocks of (16 gate rows, the 16 matching up rows): [block][gate|up][16]
             tma_load_5d_2sm(a_dst, &tmW, fb, kb * BK, 0, 0, wrow, e);
           } else {
             tma_load_2d_2sm(a_dst, &tmW, fb, kb * BK, wrow);
           }
-          if constexpr (MODE == kGemm2) {
-            int r = trow;
-            uint8_t* d = b_dst;
-#pragma unroll
-            for (int i = 0; i < kTokBoxes; ++i) {
-              const int box = kHalf >> i;
-              if (half & box) {
-                tma_load_2d_2sm(d, &tmT.m[i], fb, kb * BK, r);
-                r += box;
-                d += box * 128;
-              }
-            }
-          }
+          // GEMM2: always a whole 128-row box of token rows, whatever the chunk's N (rows
+          // past the expert's are the next expert's or the zero fill; the MMA reads N/2 of
+          // them).  Boxes sized to the chunk -- up to five per stage for a short last chunk
+          // -- measured far slower: Qwen3-30B-A3B-shaped GEMM2 255 against 205 us.
+          if constexpr (MODE == kGemm2) tma_load_2d_2sm(b_dst, &tmT, fb, kb * BK, trow);
         }
         __syncwarp();
       }
@@ -631,7 +613,7 @@ bool tmap_w13_interleaved(CUtensorMap* m, const void* ptr, int H, int I, int E) 
 constexpr int kStages = 6;
 
 template <int MODE>
-cudaError_t run_ps(const CUtensorMap& w, const TokMaps& t, const CUtensorMap& o, const PsArgs& a,
+cudaError_t run_ps(const CUtensorMap& w, const CUtensorMap& t, const CUtensorMap& o, const PsArgs& a,
                    cudaStream_t stream) {
   using Cf = PsCfg<MODE, kStages>;
   auto kern = pair_swap_gemm_kernel<MODE, kStages>;
@@ -644,24 +626,13 @@ cudaError_t run_ps(const CUtensorMap& w, const TokMaps& t, const CUtensorMap& o,
 
 }  // namespace
 
-// Tuning switch while the kernels are compared: MOE_GEMM_IMPL=old keeps the single-SM /
-// 256-row-pair kernels.
-bool use_pair_swap(const GemmProblem& p) {
-  static const bool old = [] {
-    const char* e = getenv("MOE_GEMM_IMPL");
-    return e && e[0] == 'o';
-  }();
-  return !old && p.R > 0;
-}
-
 cudaError_t launch_gemm1_pair_swap(const GemmProblem& p, const uint16_t* x,
                                    const int32_t* row2assign, const int32_t* offsets,
                                    const uint16_t* w13, uint16_t* act, int* status,
                                    cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
   const bool relu2 = p.act == 1;
-  CUtensorMap tw, to;
-  TokMaps tt{};
+  CUtensorMap tw, to, tt{};
   const bool maps = relu2 ? tmap_operand(&tw, w13, p.H, static_cast<uint64_t>(p.E) * p.I, WROWS)
                          : tmap_w13_interleaved(&tw, w13, p.H, p.I, p.E);
   if (!maps || !tmap_out(&to, act, p.I, p.R, relu2 ? 32 : 16)) return cudaErrorInvalidValue;
@@ -687,14 +658,10 @@ cudaError_t launch_gemm2_pair_swap(const GemmProblem& p, const uint16_t* act,
                                    const int32_t* offsets, const uint16_t* w2, uint16_t* y,
                                    int* status, cudaStream_t stream, int* launches) {
   if (p.R == 0) return cudaSuccess;
-  CUtensorMap tw, to;
-  TokMaps tt;
+  CUtensorMap tw, to, tt;
   if (!tmap_operand(&tw, w2, p.I, static_cast<uint64_t>(p.E) * p.H, WROWS) ||
-      !tmap_out(&to, y, p.H, p.R, 32))
+      !tmap_operand(&tt, act, p.I, p.R, kHalf) || !tmap_out(&to, y, p.H, p.R, 32))
     return cudaErrorInvalidValue;
-  for (int i = 0; i < kTokBoxes; ++i)
-    if (!tmap_operand(&tt.m[i], act, p.I, p.R, static_cast<uint32_t>(kHalf >> i)))
-      return cudaErrorInvalidValue;
   PsArgs a{};
   a.offsets = offsets;
   a.out = y;

@@ -199,9 +199,15 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     tmem_alloc(s_tmem, C::TMEM_COLS);
     tmem_relinquish();
   }
-  pdl_wait();  // the offsets (and every other input) come from earlier kernels
+  // GEMM1 reads the token rows, row2assign and the offsets in several roles: every thread
+  // waits for the kernels before it.  GEMM2's weights and expert offsets are final before
+  // the kernel just ahead of it could start (the offsets come from the front end, which had
+  // completed by then), so only its producer waits -- after issuing the weight boxes of its
+  // first ring of stages -- and the token rows (act, from GEMM1) are loaded after the wait;
+  // the weights stream while GEMM1 finishes.  The offsets are read through L2 (__ldcg).
+  if constexpr (GEMM1) pdl_wait();
   pdl_launch_dependents();  // the next kernel's CTAs may take SMs as this grid's CTAs exit
-  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldg(args.offsets + i);
+  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = __ldcg(args.offsets + i);
   __syncthreads();
   if (warp == 0) {  // token tiles of NT rows per expert
     const int per = (E + 31) / 32;
@@ -250,6 +256,22 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     uint32_t fill = 0;
     int skipped = -1;
     bool ok = true;
+    // GEMM2: token-row loads of the fills issued before the wait for the kernel ahead
+    bool waited = GEMM1;
+    int npend = 0;
+    uint32_t pend_fill[STAGES];
+    int pend_row[STAGES], pend_kb[STAGES];
+    auto flush = [&]() {
+      pdl_wait();
+      waited = true;
+      if (lane == 0)
+        for (int i = 0; i < npend; ++i) {
+          const int ps = static_cast<int>(pend_fill[i] % STAGES);
+          tma_load_2d(smem + ps * C::STAGE + C::A_BYTES, &tmT, &full[ps], pend_kb[i] * BK,
+                      pend_row[i]);
+        }
+      __syncwarp();
+    };
     for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
       int e, tt, ft, sp;
       decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
@@ -276,12 +298,19 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
           } else {
             mbar_arrive_expect_tx(&full[s], C::STAGE);
             tma_load_2d(w_dst, &tmW, &full[s], kb * BK, wrow);
-            tma_load_2d(t_dst, &tmT, &full[s], kb * BK, row0);
+            if (waited) tma_load_2d(t_dst, &tmT, &full[s], kb * BK, row0);
           }
+        }
+        if (!waited) {   // (GEMM2 only) the token rows of this fill wait for the flush
+          pend_fill[npend] = fill;
+          pend_row[npend] = row0;
+          pend_kb[npend] = kb;
+          if (++npend == STAGES) flush();   // before the ring is reused
         }
         __syncwarp();
       }
     }
+    if (!waited) flush();   // fewer fills than stages, or the loop gave up
     if (!ok && lane == 0) {
       *s_abort = 1;
       set_status(args.status, kStatusTimeout);

@@ -81,7 +81,8 @@ struct GemmProblem {
   uint64_t wait_limit_ns;
 };
 
-// Grouped GEMM1 + SwiGLU, BF16 (x gathered by row2assign, act expert-sorted).
+// Grouped GEMM1 + SwiGLU (or ReLU2), BF16 (x gathered by row2assign, act expert-sorted):
+// the decode-sized kernels for T <= 64 (SwiGLU), else the SM-pair kernels.
 cudaError_t launch_gemm1_bf16(const GemmProblem& p, const uint16_t* x, const int32_t* row2assign,
                               const int32_t* offsets, const uint16_t* w13, uint16_t* act,
                               int* status, cudaStream_t stream, int* launches);
@@ -91,21 +92,8 @@ cudaError_t launch_gemm2_bf16(const GemmProblem& p, const uint16_t* act, const i
                               const uint16_t* w2, uint16_t* y, int* status, cudaStream_t stream,
                               int* launches);
 
-// The same BF16 GEMMs on SM pairs (cta_group::2, 256-row tiles); use_pair_gemm decides
-// for GEMM2 from the average rows per expert and its K.
-bool use_pair_gemm(int64_t R, int E, int K);
-bool use_pair_gemm1(int64_t R, int E);
-cudaError_t launch_gemm1_bf16_2sm(const GemmProblem& p, const uint16_t* x,
-                                  const int32_t* row2assign, const int32_t* offsets,
-                                  const uint16_t* w13, uint16_t* act, int* status,
-                                  cudaStream_t stream, int* launches);
-cudaError_t launch_gemm2_bf16_2sm(const GemmProblem& p, const uint16_t* act,
-                                  const int32_t* offsets, const uint16_t* w2, uint16_t* y,
-                                  int* status, cudaStream_t stream, int* launches);
-
 // Large-batch BF16 GEMMs on SM pairs with the weights on the MMA's M = 256 side and
 // chunks of up to 256 token rows on its N side (gemm_pair_swap.cu).
-bool use_pair_swap(const GemmProblem& p);
 cudaError_t launch_gemm1_pair_swap(const GemmProblem& p, const uint16_t* x,
                                    const int32_t* row2assign, const int32_t* offsets,
                                    const uint16_t* w13, uint16_t* act, int* status,

@@ -5,11 +5,10 @@
 // the predecessor produces or reads.  Every kernel signals pdl_launch_dependents() right
 // after its own pdl_wait(): the successor's CTAs are then scheduled as soon as SM resources
 // free up (the persistent GEMMs' tail wave), which is safe because the successor's
-// pdl_wait() still waits for this grid's completion.  MOE_PDL=0 turns the overlap off.
+// pdl_wait() still waits for this grid's completion.
 #pragma once
 
 #include <cuda_runtime.h>
-#include <stdlib.h>
 
 #include <utility>
 
@@ -19,14 +18,6 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-inline bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("MOE_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
 }
 
 template <typename... KArgs, typename... Args>
@@ -39,7 +30,7 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);

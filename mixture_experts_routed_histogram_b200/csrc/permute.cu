@@ -471,9 +471,12 @@ __device__ bool grid_barrier(unsigned* gbar, int* s_ok, uint64_t limit_ns, unsig
       __threadfence();
       atomicAdd(gbar + 1, 1u);
     } else {
+      // poll with a short sleep between reads, so hundreds of waiting CTAs do not keep the
+      // line's L2 slice busy while the last arrivals are still on their way
       const uint64_t start = globaltimer_ns();
       for (uint32_t i = 0; *vgen == gen; ++i) {
-        if ((i & 63u) == 63u && globaltimer_ns() - start > limit_ns) {
+        __nanosleep(64);
+        if ((i & 15u) == 15u && globaltimer_ns() - start > limit_ns) {
           ok = false;
           break;
         }
@@ -515,8 +518,14 @@ __global__ void __launch_bounds__(kFusedThreads)
   pdl_launch_dependents();
   __syncthreads();
 
-  // ---- phase 1: route the block's tokens, count its assignments per expert
+  // ---- phase 1: route the block's tokens, count its assignments per expert; a warp with a
+  // second token asks for that token's logits (into L2) before routing the first
   for (int64_t t = t0 + warp; t < t1; t += kFusedWarps) {
+    if (t + kFusedWarps < t1) {
+      const float* nxt = logits + (t + kFusedWarps) * E;
+      for (int e = lane * 32; e < E; e += 32 * 32)   // one 128-byte line per lane
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + e));
+    }
     int id;
     float wt;
     route_token_warp<VPT>(logits + t * E, E, k, score, renorm, lane, id, wt);
@@ -535,22 +544,32 @@ __global__ void __launch_bounds__(kFusedThreads)
 
   bool ok = grid_barrier(gbar, &s_ok, limit_ns, inject_stall ? 1u : 0u);
 
-  // ---- phase 2: one warp per expert scans its counts over the blocks
+  // ---- phase 2: one warp per expert scans its counts over the blocks (all of a lane's
+  // loads are issued before the scan, so the warp waits for L2 about once)
   if (ok) {
+    constexpr int kPer = kFusedMaxBlocks / 32;
     for (int e = me * kFusedWarps + warp; e < Ea; e += nb * kFusedWarps) {
       const int32_t* src = cc + static_cast<int64_t>(e) * nb;
       int32_t* dst = base + static_cast<int64_t>(e) * nb;
-      int run = 0;
-      for (int c0 = 0; c0 < nb; c0 += 32) {
-        const int v = c0 + lane < nb ? __ldcg(src + c0 + lane) : 0;
-        int incl = v;
+      int v[kPer];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += y;
+      for (int i = 0; i < kPer; ++i) {
+        const int c = i * 32 + lane;
+        v[i] = c < nb ? __ldcg(src + c) : 0;
+      }
+      int run = 0;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        if (i * 32 < nb) {
+          int incl = v[i];
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+          }
+          if (i * 32 + lane < nb) dst[i * 32 + lane] = run + incl - v[i];
+          run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (c0 + lane < nb) dst[c0 + lane] = run + incl - v;
-        run += __shfl_sync(0xffffffffu, incl, 31);
       }
       if (lane == 0) tot[e] = run;
     }

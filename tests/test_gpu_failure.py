@@ -4,9 +4,9 @@ expires, every role of the kernel unwinds, the status word reads MOE_ERR_DEVICE_
 and the context stays usable: the same launch without the hook gives the same bits as a
 clean launch made before the failure (and the first case also matches the oracle).
 
-The shapes pick each GEMM kernel family: decode-sized (weights on the MMA's M side),
-single-SM tiles, SM-pair tiles (GEMM2 at >= 768 rows per expert), and the block-scaled
-FP8 x MXFP4 kernels in both their forms."""
+The shapes pick each GEMM kernel family: decode-sized (single SMs, weights on the MMA's
+M = 128 side), SM pairs (weights on the M = 256 side; SwiGLU, ReLU2 and experts of several
+256-row chunks), and the block-scaled FP8 x MXFP4 kernels in both their forms."""
 import numpy as np
 import pytest
 import torch
@@ -20,8 +20,9 @@ pytestmark = pytest.mark.gpu
 
 CASES = {
     "bf16_swap": I.WORKLOADS["tiny"],                                  # T <= 64
-    "bf16_single_sm": I.Workload("fs", 300, 256, 128, 8, 2),           # 75 rows / expert
-    "bf16_pair_gemm2": I.Workload("fp", 2048, 256, 128, 2, 1),         # 1024 rows / expert
+    "bf16_pairs": I.Workload("fs", 300, 256, 128, 8, 2),               # 75 rows / expert
+    "bf16_pairs_relu2": I.Workload("fr", 300, 256, 128, 8, 2, act="relu2"),
+    "bf16_pairs_4_chunks": I.Workload("fp", 2048, 256, 128, 2, 1),     # 1024 rows / expert
     "fp8_single_sm": I.Workload("f8", 300, 256, 256, 4, 2, dtype="fp8_mxfp4"),
     "fp8_swap": I.Workload("f8s", 64, 256, 128, 8, 2, dtype="fp8_mxfp4"),
 }

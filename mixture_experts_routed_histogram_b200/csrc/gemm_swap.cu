@@ -120,6 +120,72 @@ __device__ __forceinline__ int choose_gemm2_splits(int tiles, int kb, int smax, 
   return best;
 }
 
+__device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// The work of one CTA.  Round robin: tasks c, c + P, ... of the (expert, token tile,
+// feature tile, K slice) queue.  Stream-K (the decode GEMM2 with partial sums): the
+// (tile, K block) units of all tiles, U of them, are dealt to the first P' CTAs as equal
+// contiguous ranges [c U / P', (c+1) U / P'), cut at tile boundaries into segments; the
+// segment of tile t that CTA c holds writes partial-sum slot c - (first CTA of t), and the
+// CTA holding a tile's last K block also clears its higher slots up to the slot count the
+// combine sums, so every slot it reads is defined and the sum keeps a fixed order.
+struct SwapWork {
+  int e, tt, ft;        // expert, token tile, feature tile
+  int kb0, kb1;         // K blocks [kb0, kb1)
+  int slot;             // partial-sum slot
+  bool last;            // this segment ends the tile (stream-K: clear the higher slots)
+};
+
+struct SwapIter {
+  const int* s_tile;
+  int E, ftiles, splits, kb_all;
+  bool sk;
+  int64_t u, u_hi, U;   // stream-K range of this CTA
+  int P;                // stream-K CTAs
+  int task, total, step;  // round robin
+  __device__ __forceinline__ int owner(int64_t unit) const {   // CTA holding a unit
+    return static_cast<int>(((unit + 1) * P - 1) / U);
+  }
+  __device__ __forceinline__ bool next(SwapWork& w) {
+    int sp = 0;
+    if (sk) {
+      if (u >= u_hi) return false;
+      const int tile = static_cast<int>(u / kb_all);
+      w.kb0 = static_cast<int>(u - static_cast<int64_t>(tile) * kb_all);
+      w.kb1 = static_cast<int>(i64min(kb_all, w.kb0 + (u_hi - u)));
+      w.slot = owner(u) - owner(static_cast<int64_t>(tile) * kb_all);
+      w.last = w.kb1 == kb_all;
+      u += w.kb1 - w.kb0;
+      decode_swap(tile, s_tile, E, ftiles, 1, w.e, w.tt, w.ft, sp);
+      return true;
+    }
+    if (task >= total) return false;
+    decode_swap(task, s_tile, E, ftiles * splits, splits, w.e, w.tt, w.ft, sp);
+    const int kb_per = kb_all / splits;
+    w.kb0 = sp * kb_per;
+    w.kb1 = w.kb0 + kb_per;
+    w.slot = sp;
+    w.last = false;
+    task += step;
+    return true;
+  }
+};
+
+// CTAs that share the stream-K work: all of them, unless that leaves fewer than 24 K
+// blocks per CTA (a task switch costs about 16 K blocks of streaming) or lets one tile of
+// kb blocks span more than kMaxSplits CTAs (each CTA's range is >= ceil(kb / 15) units).
+__device__ __forceinline__ int64_t stream_k_ctas(int64_t units, int64_t kb, int grid) {
+  const int64_t min_len = i64max(24, (kb + kMaxSplits - 2) / (kMaxSplits - 1));
+  return i64max(1, i64min(grid, units / min_len));
+}
+
+// Partial-sum slots a tile of kb blocks can span when U units are dealt to P CTAs.
+__device__ __forceinline__ int stream_k_slots(int64_t U, int64_t kb, int64_t P) {
+  const int64_t len = i64max(1, U / P);   // the shortest CTA range
+  return static_cast<int>(i64min(kMaxSplits, (kb + len - 1) / len + 1));
+}
+
 __device__ __forceinline__ float silu_mul_s(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
@@ -233,11 +299,15 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     }
     if (lane == 31) {
       s_tile[E] = incl;
-      // args.splits > 1 selects the partial-sum output; GEMM2 picks its own slice count
-      *s_splits = (!GEMM1 && args.splits > 1)
-                      ? choose_gemm2_splits(incl * args.ftiles, args.K / BK, args.splits,
-                                            gridDim.x)
-                      : args.splits;
+      // args.splits > 1 selects the partial-sum output.  GEMM2 then runs stream-K; the
+      // number of partial-sum slots a tile can span (what the combine sums) is stored
+      if (!GEMM1 && args.splits > 1) {
+        const int64_t kb = args.K / BK;
+        const int64_t U = static_cast<int64_t>(incl) * args.ftiles * kb;
+        *s_splits = stream_k_slots(U, kb, stream_k_ctas(U, kb, gridDim.x));
+      } else {
+        *s_splits = args.splits;
+      }
       if (!GEMM1 && args.splits_used && blockIdx.x == 0) *args.splits_used = *s_splits;
     }
   }
@@ -246,10 +316,33 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int kb_all = args.K / BK;
-  const int splits = *s_splits;
+  const bool stream_k = !GEMM1 && args.splits > 1;
+  const int splits = stream_k ? 1 : *s_splits;   // round robin: K slices per tile
+  const int nslots = *s_splits;                   // stream-K: partial-sum slots
   const int per_tile = args.ftiles * splits;
   const int total = s_tile[E] * per_tile;
   const int kb_per = kb_all / splits;
+  auto make_iter = [&]() {
+    SwapIter it{};
+    it.s_tile = s_tile;
+    it.E = E;
+    it.ftiles = args.ftiles;
+    it.splits = splits;
+    it.kb_all = kb_all;
+    it.sk = stream_k;
+    if (stream_k) {
+      it.U = static_cast<int64_t>(s_tile[E]) * args.ftiles * kb_all;
+      it.P = static_cast<int>(stream_k_ctas(it.U, kb_all, gridDim.x));
+      const int c = static_cast<int>(blockIdx.x);
+      it.u = c < it.P ? static_cast<int64_t>(c) * it.U / it.P : it.U;
+      it.u_hi = c < it.P ? static_cast<int64_t>(c + 1) * it.U / it.P : it.U;
+    } else {
+      it.task = blockIdx.x;
+      it.total = total;
+      it.step = gridDim.x;
+    }
+    return it;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -272,12 +365,13 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
         }
       __syncwarp();
     };
-    for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
-      int e, tt, ft, sp;
-      decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
+    SwapIter it = make_iter();
+    SwapWork wk;
+    while (ok && it.next(wk)) {
+      const int e = wk.e, tt = wk.tt, ft = wk.ft;
       const int row0 = s_off[e] + tt * NT;
       const int wrow = GEMM1 ? e * args.b_rows + ft * 64 : e * args.b_rows + ft * BMW;
-      for (int kb = sp * kb_per; kb < (sp + 1) * kb_per; ++kb, ++fill) {
+      for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++fill) {
         const int s = fill % STAGES;
         const uint32_t ph = (fill / STAGES) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, s_abort, lim))) {
@@ -324,7 +418,9 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     if (lane == 0) {
       uint32_t fill = 0, tc = 0;
       bool ok = true;
-      for (int task = blockIdx.x; task < total && ok; task += gridDim.x) {
+      SwapIter it = make_iter();
+      SwapWork wk;
+      while (ok && it.next(wk)) {
         const int acc = tc & 1;
         const uint32_t aph = (tc >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, s_abort, lim)) {
@@ -333,7 +429,7 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NT);
-        for (int kb = 0; kb < kb_per; ++kb, ++fill) {
+        for (int kb = 0; kb < wk.kb1 - wk.kb0; ++kb, ++fill) {
           const int s = fill % STAGES;
           const uint32_t ph = (fill / STAGES) & 1u;
           if (!mbar_wait(&full[s], ph, s_abort, lim)) {
@@ -409,9 +505,10 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
     const int q = warp & 3;          // TMEM lanes 32q..32q+31 = weight rows of the tile
     uint32_t tc = 0;
     bool ok = true;
-    for (int task = blockIdx.x; task < total; task += gridDim.x) {
-      int e, tt, ft, sp;
-      decode_swap(task, s_tile, E, per_tile, splits, e, tt, ft, sp);
+    SwapIter it = make_iter();
+    SwapWork wk;
+    while (it.next(wk)) {
+      const int e = wk.e, tt = wk.tt, ft = wk.ft, sp = wk.slot;
       const int row0 = s_off[e] + tt * NT;
       const int rows = min(NT, s_off[e + 1] - row0);
       const int acc = tc & 1;
@@ -470,6 +567,12 @@ __global__ void __launch_bounds__(SwapCfg<GEMM1, NT, STAGES>::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < NT; ++c)
             if (c < rows) dst[static_cast<int64_t>(row0 + c) * args.n_out + o] = __uint_as_float(v[c]);
+          if (wk.last)   // stream-K: the tile's unused higher slots read as zeros
+            for (int z = sp + 1; z < nslots; ++z) {
+              float* zd = args.part + static_cast<int64_t>(z) * args.R * args.n_out;
+              for (int c = 0; c < rows; ++c)
+                zd[static_cast<int64_t>(row0 + c) * args.n_out + o] = 0.0f;
+            }
         } else {
 #pragma unroll
           for (int c = 0; c < NT; ++c)

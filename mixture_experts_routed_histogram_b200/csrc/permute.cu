@@ -399,9 +399,12 @@ cudaError_t launch_route_permute_small(const float* logits, int64_t T, int E, in
 //            shared memory and count the CTA's assignments per expert -> cc[e][b];
 //   barrier  grid-wide: an arrival count and a generation word in the workspace's status
 //            block, bounded wait;
-//   phase 2  every CTA sums cc over all blocks itself (tot[e]) and over the blocks before
-//            it (base[e]) -- integer sums, so the order does not matter -- scans tot over
-//            the experts (offsets; CTA 0 writes counts and offsets) and scatters its
+//   phase 2  tot[e] (all blocks' counts) and base[e] (those of the blocks before this
+//            one): with few experts x blocks (<= 32768 cells) every CTA sums cc itself --
+//            integer sums, so the order does not matter; with more, one warp per expert
+//            (spread over the CTAs) scans its row of cc into base and tot in global memory
+//            and a second barrier precedes the reads.  Then each CTA scans tot over the
+//            experts (offsets; CTA 0 writes counts and offsets) and scatters its
 //            assignments in order with the warp-match and round-stamp ranking of
 //            scatter_kernel: row = offsets[e] + #{a' < a : ids[a'] == e}.
 // Each step waits on global memory about once.  At T = 8192, E = 128, k = 8 the kernel takes
@@ -415,6 +418,7 @@ constexpr int kFusedThreads = 1024;
 constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kFusedMaxBlocks = 1024;
 constexpr int kFusedIdsSmem = 8192;   // assignments of a CTA kept in shared memory
+constexpr int64_t kSinglePassCells = 32768;   // experts x blocks summed by every CTA itself
 
 int fused_blocks_cap(int64_t T) {
   return static_cast<int>(std::min<int64_t>((T + kFusedWarps - 1) / kFusedWarps, kFusedMaxBlocks));
@@ -500,6 +504,7 @@ __global__ void __launch_bounds__(kFusedThreads)
     route_permute_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int ns,
                          int score, int renorm, int tpc, int32_t* __restrict__ ids,
                          float* __restrict__ w, int32_t* __restrict__ cc,
+                         int32_t* __restrict__ base, int32_t* __restrict__ tot,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ row2assign, int32_t* __restrict__ assign2row,
                          unsigned* gbar, int* status, uint64_t limit_ns, int inject_stall) {
@@ -563,31 +568,75 @@ __global__ void __launch_bounds__(kFusedThreads)
     return;
   }
 
-  // ---- phase 2: tot[e] = all blocks' counts, base[e] = those of the blocks before this
-  // one; a group of g lanes (a power of two, g * Ea <= kFusedThreads when Ea is small)
-  // shares an expert's row of cc, every load issued before the sums
-  int g = 1;
-  while (g < 32 && 2 * g * Ea <= kFusedThreads) g *= 2;
-  const int per_warp = 32 / g;   // experts a warp handles per pass (the loop is warp-uniform)
-  for (int eb = warp * per_warp; eb < Ea; eb += kFusedWarps * per_warp) {
-    const int e0 = eb + lane / g, sub = lane & (g - 1);
-    int all = 0, before = 0;
-    if (e0 < Ea) {
-      const int32_t* row = cc + static_cast<int64_t>(e0) * nb;
+  // ---- phase 2: tot[e] = all blocks' counts, base[e] = those of the blocks before this one
+  if (static_cast<int64_t>(Ea) * nb <= kSinglePassCells) {
+    // few cells: every CTA sums them itself; a group of g lanes (a power of two, g * Ea <=
+    // kFusedThreads when Ea is small) shares an expert's row of cc, every load issued
+    // before the sums
+    int g = 1;
+    while (g < 32 && 2 * g * Ea <= kFusedThreads) g *= 2;
+    const int per_warp = 32 / g;   // experts a warp handles per pass (the loop is warp-uniform)
+    for (int eb = warp * per_warp; eb < Ea; eb += kFusedWarps * per_warp) {
+      const int e0 = eb + lane / g, sub = lane & (g - 1);
+      int all = 0, before = 0;
+      if (e0 < Ea) {
+        const int32_t* row = cc + static_cast<int64_t>(e0) * nb;
 #pragma unroll 8
-      for (int c = sub; c < nb; c += g) {
-        const int v = __ldcg(row + c);
-        all += v;
-        before += c < me ? v : 0;
+        for (int c = sub; c < nb; c += g) {
+          const int v = __ldcg(row + c);
+          all += v;
+          before += c < me ? v : 0;
+        }
+      }
+      for (int off = g >> 1; off > 0; off >>= 1) {
+        all += __shfl_xor_sync(0xffffffffu, all, off);
+        before += __shfl_xor_sync(0xffffffffu, before, off);
+      }
+      if (e0 < Ea && sub == 0) {
+        hist[e0] = all;
+        cursor[e0] = before;
       }
     }
-    for (int off = g >> 1; off > 0; off >>= 1) {
-      all += __shfl_xor_sync(0xffffffffu, all, off);
-      before += __shfl_xor_sync(0xffffffffu, before, off);
+  } else {
+    // many cells (many experts): one warp per expert, spread over the CTAs, scans its row of
+    // cc into base[e][*] and tot[e]; after a second barrier each CTA reads its column
+    constexpr int kPer = kFusedMaxBlocks / 32;
+    for (int e = warp * nb + me; e < Ea; e += nb * kFusedWarps) {
+      const int32_t* src = cc + static_cast<int64_t>(e) * nb;
+      int32_t* dst = base + static_cast<int64_t>(e) * nb;
+      int v[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int c = i * 32 + lane;
+        v[i] = c < nb ? __ldcg(src + c) : 0;
+      }
+      int run = 0;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        if (i * 32 < nb) {
+          int incl = v[i];
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+          }
+          if (i * 32 + lane < nb) dst[i * 32 + lane] = run + incl - v[i];
+          run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      if (lane == 0) tot[e] = run;
     }
-    if (e0 < Ea && sub == 0) {
-      hist[e0] = all;
-      cursor[e0] = before;
+    if (!grid_barrier(gbar, &s_ok, limit_ns, 0u)) {
+      if (tid == 0) set_status(status, kStatusTimeout);
+      for (int e = tid; e <= Ea; e += kFusedThreads) {
+        offsets[e] = 0;
+        if (e < Ea) counts[e] = 0;
+      }
+      return;
+    }
+    for (int e = tid; e < Ea; e += kFusedThreads) {
+      hist[e] = __ldcg(tot + e);
+      cursor[e] = __ldcg(base + static_cast<int64_t>(e) * nb + me);
     }
   }
   __syncthreads();
@@ -629,7 +678,7 @@ __global__ void __launch_bounds__(kFusedThreads)
 }
 
 size_t route_permute_scratch_bytes(int64_t T, int E) {
-  return static_cast<size_t>(E) * fused_blocks_cap(T) * sizeof(int32_t);
+  return (static_cast<size_t>(2) * E * fused_blocks_cap(T) + E) * sizeof(int32_t);
 }
 
 template <int VPT>
@@ -659,6 +708,8 @@ cudaError_t launch_fused(const float* logits, int64_t T, int E, int k, int ns, i
       fixed + sizeof(int) * static_cast<size_t>(std::min<int64_t>(static_cast<int64_t>(tpc) * ks,
                                                                    kFusedIdsSmem));
   int32_t* cc = scratch;
+  int32_t* base = cc + static_cast<int64_t>(Ea) * nb_used;
+  int32_t* tot = base + static_cast<int64_t>(Ea) * nb_used;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nb_used);
   cfg.blockDim = dim3(kFusedThreads);
@@ -671,8 +722,8 @@ cudaError_t launch_fused(const float* logits, int64_t T, int E, int k, int ns, i
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, logits, T, E, k, ns, score, renorm, tpc, ids, w, cc,
-                            counts, offsets, row2assign, assign2row, gbar, status, limit_ns,
+  return cudaLaunchKernelEx(&cfg, kern, logits, T, E, k, ns, score, renorm, tpc, ids, w, cc, base,
+                            tot, counts, offsets, row2assign, assign2row, gbar, status, limit_ns,
                             g_inject_stall);
 }
 

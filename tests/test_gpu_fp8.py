@@ -167,3 +167,34 @@ def test_forward_fp8_full_size(T):
     checks a seeded 256-token subset that always includes the first and last token."""
     wl = W["fp8_mxfp4"].with_T(T)
     _forward_check(wl, I.parity_tokens(T, 256))
+
+
+@pytest.mark.parametrize("T", [64, 300])
+def test_forward_fp8_on_quantised_gaussian_weights(T):
+    """The block-scaled forward on MXFP4 weights that the oracle's OCP MX quantiser made from
+    N(0, 1/fan_in) bf16 weights (the synthetic generator draws codes and scale bytes
+    directly, with a narrower spread of scales): both sides consume the same codes."""
+    wl16 = I.Workload("qg", T, 256, 256, 8, 2)
+    wl = I.Workload("qg", T, 256, 256, 8, 2, dtype="fp8_mxfp4")
+    x = I.make_x(wl16, 0, "cpu")
+    logits = I.make_logits(wl16, x)
+    w13_bf, w2_bf = I.make_weights(wl16, 0, "cpu")
+    w13p, w13sf = oracle.quant_mxfp4(I.bits(w13_bf))
+    w2p, w2sf = oracle.quant_mxfp4(I.bits(w2_bf))
+    # scale bytes as gaussian blocks give them (three values here) and codes that are not
+    # drawn from the generator's table
+    assert len(np.unique(w13sf)) >= 3 and len(np.unique(w2sf)) >= 3
+    shape = C.MoeShape.from_workload(wl)
+    ws = workspace(shape)
+    buf, out = with_canary(T, wl.H)
+    d = {n: torch.from_numpy(np.ascontiguousarray(a)).to(dev())
+         for n, a in (("w13", w13p), ("w13_sf", w13sf), ("w2", w2p), ("w2_sf", w2sf))}
+    C.moe_forward(shape, x.to(dev()), logits.to(dev()), d["w13"], d["w13_sf"], d["w2"],
+                  d["w2_sf"], out, None, ws)
+    torch.cuda.synchronize()
+    assert C.moe_get_device_status(ws) == 0
+    assert canary_intact(buf, T, wl.H)
+    oids, ow = oracle_route(wl, logits)
+    ref, _ = oracle.forward_fp8_mxfp4(I.bits(x), oids, ow, w13p, w13sf, w2p, w2sf,
+                                      np.arange(T), requant_act=True)
+    assert_close(f64(out), ref, COS_FP8, what=f"fp8 forward on quantised gaussian weights T={T}")

@@ -45,18 +45,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # The block-scaled e4m3 x e2m1 MMA is taken to run at this FP8 rate.
 FP8_PEAKS = {"fp8_tflops": 3094.9, "fp8_tflops_sustained": 2543.3}
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernels, from the ncu captures summarised in profiles/ (the DRAM-bytes pass of
-# dram_traffic_current_kernels, and gemm_mx_fp8_mxfp4_T8192); an entry is removed when its
-# kernel changes after the capture.
+# kernels, from the ncu captures summarised in profiles/dram_traffic_current_kernels.md
+# (decode: both GEMMs from the one --set full capture in profiles/gemm_swap_decode_T1.md);
+# an entry is removed when its kernel changes after the capture.
 NCU_TRAFFIC = {
-    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 969.10e6 + 90.88e6,
-    ("qwen3_30b_a3b", 8192, "gemm2"): 503.43e6 + 236.24e6,     # SM-pair kernel
-    ("decode", 1, "gemm1_swiglu"): 469.835e6 + 0.470e6,
-    ("decode", 1, "gemm2"): 234.996e6 + 0.255e6,
-    ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.745e6 + 1.250e6,
-    ("fp8_mxfp4", 128, "gemm2"): 446.548e6 + 5.579e6,
-    ("fp8_mxfp4", 8192, "gemm1_swiglu"): 1180.74e6 + 55.53e6,
-    ("fp8_mxfp4", 8192, "gemm2"): 500.67e6 + 380.47e6,
+    ("qwen3_30b_a3b", 8192, "gemm1_swiglu"): 975.80e6 + 92.60e6,   # pair_swap_gemm_kernel
+    ("qwen3_30b_a3b", 8192, "gemm2"): 503.60e6 + 238.20e6,
+    ("decode", 1, "gemm1_swiglu"): 469.82e6 + 4.57e6,             # swap_gemm_bf16_kernel
+    ("decode", 1, "gemm2"): 236.18e6 + 4.58e6,                    # (stream-K)
+    ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.80e6 + 2.60e6,        # mx_swap_gemm_kernel
+    ("fp8_mxfp4", 128, "gemm2"): 446.60e6 + 5.50e6,
+    ("fp8_mxfp4", 8192, "gemm1_swiglu"): 1176.10e6 + 50.60e6,     # mx_grouped_gemm_kernel
+    ("fp8_mxfp4", 8192, "gemm2"): 499.90e6 + 376.40e6,
 }
 
 

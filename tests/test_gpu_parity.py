@@ -265,9 +265,9 @@ def test_forward_full_size_parity(name):
 # Expert row counts that put an expert's last token chunk (of up to 256 rows, padded to a
 # multiple of 16) on every boundary: 1, 15-17, 31-33 rows, exactly one and two chunks, one
 # row more or less, experts of three to seven chunks (767 .. 1537), and empty experts
-# between them.
+# between them; and last chunks of 17-65 rows after two or three full ones (273 .. 788).
 CHUNK_COUNTS = [1, 0, 15, 16, 17, 31, 32, 33, 0, 255, 256, 257, 511, 512, 513, 8,
-                767, 768, 769, 1024, 1025, 1537]
+                767, 768, 769, 1024, 1025, 1537, 273, 530, 545, 576, 577, 788]
 
 
 def _chunk_ids():

@@ -15,10 +15,15 @@
 //          which write act = silu(g)*u for the tile's 64 features of each token row.  With
 //          K split (slice count set on the host), it writes fp32 gate|up partial sums and
 //          swiglu_parts_kernel finishes act.
-//   GEMM2: 128 output features; K (= I) may be split into S slices whose fp32 partial sums
-//          go to a workspace that the split-aware combine adds up, so that even one token
-//          (two experts) spreads its weights over every SM.  S is chosen in the kernel from
-//          the busy tiles (choose_gemm2_splits) and stored for the combine.
+//   GEMM2: 128 output features; with partial sums (the forward's decode path) it runs
+//          stream-K: the (tile, K block) units of the busy tiles, counted on the device, are
+//          cut into one contiguous range per SM, so that even one token (two experts)
+//          streams its weights on every SM.  A range's piece of a tile writes fp32 partial
+//          sums to slot j = its index among the tile's pieces (the last piece zero-fills the
+//          slots after it); the slot count goes to a workspace word and the split-aware
+//          combine adds the slots in order.  (The same split for GEMM1 measured no faster:
+//          with the weights streaming from HBM, SMs that finish early do not matter while
+//          the others still saturate it.)
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -90,34 +95,6 @@ __device__ __forceinline__ void decode_swap(int task, const int* s_tile, int E, 
   const int rest = local - tt * per_tile;
   ft = rest / splits;
   sp = rest - ft * splits;
-}
-
-// K slices for the decode-sized GEMM2, chosen on the device from the exact count of busy
-// (expert, token tile, feature tile) tiles, so that skewed routing (fewer busy experts than
-// min(E, R)) is seen.  Cost model, fitted to the decode workload (T = 1, 8, 32, 64): tasks
-// are dealt round-robin, so the CTAs work in rounds of up to P tasks of kb/s K blocks each;
-// one CTA alone streams only about 1/(0.75 P) of HBM bandwidth, so a round with a CTAs busy
-// takes kb/s * max(1, a / (0.75 P)) block times, and every round adds about 16 more (a task
-// switch measured that costly).  Candidates keep >= 24 K blocks per slice.
-__device__ __forceinline__ int choose_gemm2_splits(int tiles, int kb, int smax, int P) {
-  const float psat = 0.75f * static_cast<float>(P);
-  int best = 1;
-  float best_cost = 3.0e38f;
-  for (int s = 1; s <= smax; ++s) {
-    if (kb % s != 0 || (s > 1 && kb / s < 24)) continue;
-    const int n = tiles * s;
-    const int full = n / P, rem = n - full * P;
-    const float len = static_cast<float>(kb / s);
-    const float cost =
-        len * (static_cast<float>(full) * fmaxf(1.0f, static_cast<float>(P) / psat) +
-               (rem ? fmaxf(1.0f, static_cast<float>(rem) / psat) : 0.0f)) +
-        16.0f * static_cast<float>(full + (rem ? 1 : 0));
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
 }
 
 __device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }

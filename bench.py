@@ -55,8 +55,8 @@ NCU_TRAFFIC = {
     ("decode", 1, "gemm2"): 236.18e6 + 4.58e6,                    # (stream-K)
     ("fp8_mxfp4", 128, "gemm1_swiglu"): 891.80e6 + 2.60e6,        # mx_swap_gemm_kernel
     ("fp8_mxfp4", 128, "gemm2"): 446.60e6 + 5.50e6,
-    ("fp8_mxfp4", 8192, "gemm1_swiglu"): 1176.10e6 + 50.60e6,     # mx_grouped_gemm_kernel
-    ("fp8_mxfp4", 8192, "gemm2"): 499.90e6 + 376.40e6,
+    ("fp8_mxfp4", 8192, "gemm1_swiglu"): 924.00e6 + 50.50e6,      # mx_grouped_gemm_kernel
+    ("fp8_mxfp4", 8192, "gemm2"): 499.80e6 + 377.30e6,
 }
 
 

@@ -410,7 +410,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const uint16_t* x, const floa
     g_timer.mark(stream, "gemm2");
   } else if (moe::use_swap_gemm(T) && shape->H % 128 == 0) {
     // decode-sized: weights on the MMA's M side; GEMM2 splits K and the combine adds the
-    // partial sums.  (GEMM1 with ReLU2 runs on the single-SM kernel.)
+    // partial sums.  (GEMM1 with ReLU2 runs on the SM-pair kernel at every batch size.)
     const int splits = moe::swap_splits(p);
     float* part = at<float>(ws, L.part);  // GEMM1's partials are consumed before GEMM2's
     if (p.act == MOE_ACT_RELU2)

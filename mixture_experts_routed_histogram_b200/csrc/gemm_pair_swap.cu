@@ -17,9 +17,12 @@
 // Why this shape on B200.  A tcgen05 pair MMA (cta_group::2, M = 256) reads the N-side
 // operand half from each CTA, so per SM and per K = 64 step the ring moves 16 KB of weights
 // plus at most 16 KB of token rows for a 128 x 256 x 64 block of MMA work -- a third less
-// than the 48 KB of a single-SM 128 x 256 tile, which is what bounds the single-SM kernels
-// (operand delivery through L2).  And because N may be any multiple of 16 up to 256, an
-// expert's last chunk is padded to 16 rows, not to a 128- or 256-row tile.
+// than the 48 KB of a single-SM 128 x 256 tile.  Filling shared memory and the MMA's
+// operand reads set the pace of both, not the tensor pipe: timing-only copies of this
+// kernel took 0.65x the time with no MMAs and reached ~1.58 PFLOP/s on the tensor pipe with
+// every MMA issued twice, while one 256-token MMA set per 32 KB stage runs at ~716 SM clocks
+// against 512 of MMA work.  And because N may be any multiple of 16 up to 256, an expert's
+// last chunk is padded to 16 rows, not to a 128- or 256-row tile.
 //
 // Tasks: (expert e, feature tile ft, token chunk c), chunk-fastest, so the pairs running at
 // the same time share each weight tile through L2.  Chunk c covers sorted rows

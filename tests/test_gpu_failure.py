@@ -7,6 +7,8 @@ clean launch made before the failure (and the first case also matches the oracle
 The shapes pick each GEMM kernel family: decode-sized (single SMs, weights on the MMA's
 M = 128 side), SM pairs (weights on the M = 256 side; SwiGLU, ReLU2 and experts of several
 256-row chunks), and the block-scaled FP8 x MXFP4 kernels in both their forms."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -79,12 +81,17 @@ def test_injected_stall_reports_timeout_and_context_survives(case, which):
     clean = _run(wl, st, which).clone()
     torch.cuda.synchronize()
     assert C.moe_get_device_status(st["ws"]) == 0
-    C.moe_debug_set_wait_limit_ns(50_000_000)
+    limit_s = 0.05
+    C.moe_debug_set_wait_limit_ns(int(limit_s * 1e9))
     C.moe_debug_inject_stall(True)
     try:
+        t0 = time.perf_counter()
         _run(wl, st, which)
         torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
         assert C.moe_get_device_status(st["ws"]) == C.MOE_ERR_DEVICE_TIMEOUT
+        # every role (in SM pairs, both CTAs) unwinds within a few limits, not one per wait
+        assert elapsed < 10 * limit_s, f"stalled launch took {elapsed:.3f} s"
     finally:
         C.moe_debug_inject_stall(False)
         C.moe_debug_set_wait_limit_ns(0)
